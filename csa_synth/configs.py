@@ -1,0 +1,102 @@
+"""Workload shapes of the CSA2 sparse-attention step (synthetic, seeded).
+
+Five workloads, from a tiny decode step to a 1M-token prefill chunk:
+
+* ``tiny_decode``      - B1, 1 query, T=4096, 16 heads, indexer 4x64, K=256.
+* ``decode_64k``       - B8, T=65536, 64 heads, indexer 8x64, K=2048, 1% outlier
+                         channels x20 in the latents.
+* ``stack_128k``       - B32, T=131072, three layers Full / Reindex / Reuse.
+* ``hier_1m``          - B4, T=2^20, Full layer builds a 2048-block x 8-position
+                         candidate pool, three Reindex layers score only the pool;
+                         planted high-score keys every ~4096 positions.
+* ``prefill_1m``       - 4096 causal queries whose last one sits at position
+                         2^20 - 1 (prefix 1,044,480), bf16 latents.
+
+All share latent width D=512 (448 nope + 64 rope, stored as one latent), indexer
+head dim 64, window 128, softmax scale 1/sqrt(512).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+FULL, REINDEX, REUSE = 0, 1, 2
+
+
+@dataclass(frozen=True)
+class LayerSpec:
+    mode: int                 # FULL / REINDEX / REUSE
+    owner: int                # layer whose main KV and indexer keys this layer reads
+    reuse_from: int = -1      # REUSE: layer whose Top-K indices are reused
+    build_pool: bool = False  # FULL: also build the hierarchical candidate pool
+    pool_from: int = -1       # REINDEX: score only the pool built by this layer
+
+
+@dataclass(frozen=True)
+class Config:
+    name: str
+    B: int
+    T: int                    # cache length (positions 0..T-1), incl. the n_q new tokens
+    H: int                    # attention query heads
+    H_I: int                  # indexer heads
+    K: int                    # Top-K
+    seed: int
+    layers: List[LayerSpec] = field(default_factory=lambda: [LayerSpec(FULL, 0)])
+    n_q: int = 1              # query tokens per sequence (1 = decode)
+    D: int = 512
+    d_I: int = 64
+    W: int = 128
+    pool_blocks: int = 2048
+    pool_block_len: int = 8
+    outliers: bool = False    # 1% of latent channels x20
+    outlier_gain: float = 20.0
+    planted: bool = False     # planted high-score keys every ~4096 positions
+    plant_stride: int = 4096
+    bf16_latents: bool = False
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def n_win(self) -> int:
+        """Window entries each query attends to."""
+        return min(self.W, self.T)
+
+    @property
+    def win_rows(self) -> int:
+        """Rows in a layer's window buffer: query t reads rows [t, t + n_win)."""
+        return self.n_q + self.n_win - 1
+
+    @property
+    def owners(self) -> List[int]:
+        return sorted({l.owner for l in self.layers})
+
+    def replace(self, **kw) -> "Config":
+        return dataclasses.replace(self, **kw)
+
+
+CONFIGS = {
+    "tiny_decode": Config(name="tiny_decode", B=1, T=4096, H=16, H_I=4, K=256, seed=0),
+    "decode_64k": Config(name="decode_64k", B=8, T=65536, H=64, H_I=8, K=2048, seed=1,
+                         outliers=True),
+    "stack_128k": Config(
+        name="stack_128k", B=32, T=131072, H=64, H_I=8, K=2048, seed=2,
+        layers=[LayerSpec(FULL, 0), LayerSpec(REINDEX, 0),
+                LayerSpec(REUSE, 0, reuse_from=1)]),
+    "hier_1m": Config(
+        name="hier_1m", B=4, T=1 << 20, H=64, H_I=8, K=2048, seed=3, planted=True,
+        layers=[LayerSpec(FULL, 0, build_pool=True),
+                LayerSpec(REINDEX, 0, pool_from=0),
+                LayerSpec(REINDEX, 0, pool_from=0),
+                LayerSpec(REINDEX, 0, pool_from=0)]),
+    "prefill_1m": Config(name="prefill_1m", B=1, T=1 << 20, H=64, H_I=8, K=2048, seed=4,
+                         n_q=4096, bf16_latents=True),
+}
+
+
+def get_config(name: str, **overrides) -> Config:
+    cfg = CONFIGS[name]
+    return cfg.replace(**overrides) if overrides else cfg

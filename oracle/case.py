@@ -1,0 +1,57 @@
+"""Oracle-side encoding of the seeded synthetic workloads.
+
+Takes the fp32 values drawn by ``csa_synth`` and encodes them with this
+package's own quantisers, so that every stored byte the oracle compares
+against is produced without the CUDA path.
+"""
+from __future__ import annotations
+
+from functools import lru_cache
+
+import numpy as np
+
+from csa_synth import workload as wl
+from csa_synth.configs import Config
+
+from .quant import fp4_quant_rows, fp8_window_quant_rows, e4m3_cast
+from .layers import LayerInputs, run_stack
+
+
+class SynthCase:
+    """Encoded inputs of one sequence ``b`` of a config (rows built on demand)."""
+
+    def __init__(self, cfg: Config, b: int, sinks: bool = False, threads: int = 4):
+        self.cfg = cfg
+        self.b = b
+        self.sinks = sinks
+        self.threads = threads
+        self._keys = {}
+
+    def keys(self, owner: int) -> np.ndarray:
+        if owner not in self._keys:
+            x = wl.index_key(self.cfg, owner, self.b, 0, self.cfg.T, threads=self.threads)
+            self._keys[owner] = e4m3_cast(x)
+        return self._keys[owner]
+
+    def main_entries(self, owner: int, positions: np.ndarray) -> np.ndarray:
+        return fp4_quant_rows(wl.main_latent_at(self.cfg, owner, self.b, positions))
+
+    def main_range(self, owner: int, t0: int, n: int) -> np.ndarray:
+        return fp4_quant_rows(wl.main_latent(self.cfg, owner, self.b, t0, n, threads=self.threads))
+
+    def inputs(self, layer: int) -> LayerInputs:
+        c = self.cfg
+        return LayerInputs(
+            qI=e4m3_cast(wl.index_query(c, layer, self.b)),
+            w=wl.index_weight(c, layer, self.b),
+            q=wl.attn_query(c, layer, self.b),
+            window=fp8_window_quant_rows(wl.window_latent(c, layer, self.b)),
+            sink=wl.sink(c, layer) if self.sinks else None,
+        )
+
+    def run(self, queries=None, keep_scores=False):
+        c = self.cfg
+        return run_stack(c.layers, c.T, c.n_q, c.K, c.n_win, c.softmax_scale,
+                         self.keys, self.main_entries, self.inputs, queries=queries,
+                         pool_blocks=c.pool_blocks, pool_block_len=c.pool_block_len,
+                         keep_scores=keep_scores)
