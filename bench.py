@@ -1,0 +1,375 @@
+"""Benchmark of the CSA2 compressed sparse-attention decode step.
+
+Workload (default): ``hier_1m`` - 4 sequences at a 1,048,576-token FP4 cache,
+64 query heads, indexer 8 x 64 FP8, Top-K 2048, window 128; a Full layer that
+scores all positions and builds the 2048-block x 8-position candidate pool,
+then three Reindex layers that score only the pool.  One step = one decode
+token through the whole stack (append-encode of the new token's FP4 / FP8
+entries, indexer scores, Top-K, pool, attention) via ``csa_layer_step``.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own
+sequences (replicas, weak scaling) and the step time is the max over ranks.
+``--impl reference`` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "hier_1m"
+METRIC = "decode sparse-attn tokens/s and achieved HBM GB/s vs peak at 1M ctx, FP4 KV"
+FLUSH_BYTES = 256 << 20          # > 126 MB L2
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def _algorithmic_bytes(cfg):
+    """HBM bytes a step must move (indexer keys + selected FP4 entries + window)."""
+    per_layer_sel = cfg.B * cfg.K * 288
+    per_layer_win = cfg.B * cfg.n_win * 528
+    keys = 0
+    for L in cfg.layers:
+        if L.mode == 2:
+            continue
+        if L.pool_from >= 0:
+            keys += cfg.B * cfg.pool_blocks * cfg.pool_block_len * 64
+        else:
+            keys += cfg.B * cfg.T * 64
+    return keys + len(cfg.layers) * (per_layer_sel + per_layer_win)
+
+
+def _traffic_record(kernel_src):
+    """(bytes per launch, sha) from the committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "index_score_decode_hier_1m.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
+    h = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", txt)
+    if not m or not h:
+        return None
+    sha = hashlib.sha1(open(kernel_src, "rb").read()).hexdigest()
+    return int(m.group(1)) if h.group(1) == sha else None
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "_build", f"clocks_{os.getpid()}.csv")
+
+    def start(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- reference --
+def _oracle_case(cfg):
+    """Oracle inputs for sequence 0, prepared outside any timing: encoded keys
+    of every owner, the fp32 main latents of every position (the oracle encodes
+    the rows a step gathers on demand), each layer's own tensors."""
+    from oracle.case import SynthCase
+    from oracle import quant as oq
+    from csa_synth import workload as wl
+    nt = os.cpu_count() or 1
+    case = SynthCase(cfg, 0, threads=nt)
+    lat = {}
+    for o in cfg.owners:
+        case.keys(o)
+        lat[o] = wl.main_latent(cfg, o, 0, 0, cfg.T, threads=nt)
+    case.main_entries = lambda owner, pos: oq.fp4_quant_rows(lat[owner][pos])
+    inputs = [case.inputs(li) for li in range(len(cfg.layers))]
+    case.inputs = lambda li: inputs[li]
+    return case
+
+
+def _time_oracle(case, n_runs, budget_s=None):
+    from threadpoolctl import threadpool_limits
+    times = []
+    t_end = None if budget_s is None else time.perf_counter() + budget_s
+    with threadpool_limits(1):
+        while len(times) < n_runs:
+            t0 = time.perf_counter()
+            case.run()
+            times.append(time.perf_counter() - t0)
+            if t_end is not None and time.perf_counter() > t_end:
+                break
+    return times
+
+
+def run_reference(args, cfg, rank, world):
+    """The CPU oracle as it stands, on the host cores: each step is one
+    sequence's decode token through the whole layer stack."""
+    if rank != 0:
+        return
+    case = _oracle_case(cfg)
+    _time_oracle(case, args.warmup)
+    times = _time_oracle(case, args.steps)
+    ms = 1e3 * sum(times) / len(times)
+    v = 1e3 / ms
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "B_timed": 1, "T": cfg.T, "H": cfg.H, "H_I": cfg.H_I,
+                   "K": cfg.K, "W": cfg.W, "layers": "Full+pool(2048x8), 3x Reindex-in-pool"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": "sequence 0 of the workload per step (one decode token, all layers)"},
+        "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(cfg, seconds_budget=30.0):
+    """Oracle timed on one sequence's whole decode step (inputs prepared beforehand)."""
+    case = _oracle_case(cfg)
+    times = _time_oracle(case, 3, budget_s=seconds_budget)
+    s = min(times)
+    return {"value": round(1.0 / s, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"sequence 0 of {WORKLOAD}: one decode token through all {len(cfg.layers)} layers "
+                      f"(best of {len(times)} runs, {s:.2f} s each)"}
+
+
+# ---------------------------------------------------------------------- gpu --
+def run_gpu(args, cfg, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import indexer_selected_sparse_csa2_b200 as csa
+    from csa_synth.device import DeviceCase
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    dc = DeviceCase(cfg, device=dev)
+    descs = dc.layer_descs(append_rows=True)
+    ws_bytes = csa.csa_layer_workspace_size(descs)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        csa.csa_layer_step(descs, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- device-timed steps (L2 flushed between steps, outside the events)
+    clocks = Clocks(local_rank)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    csa.profile_enable(True)
+    n0 = csa.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    launches = csa.launch_count() - n0
+    csa.profile_enable(False)
+    kernels = csa.profile_collect()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(step_ms) / len(step_ms)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # ---- end to end through the public call: per-step inputs from pinned host
+    # memory, the step, outputs back to pinned host memory
+    h2d_pairs, d2h_pairs = [], []
+    for li, L in enumerate(cfg.layers):
+        dl = dc.layers[li]
+        for tdev in (dl.q, dl.qI, dl.w):
+            h2d_pairs.append((tdev.cpu().pin_memory(), tdev))
+        d2h_pairs.append((torch.empty_like(dl.out, device="cpu").pin_memory(), dl.out))
+        d2h_pairs.append((torch.empty_like(dl.lse, device="cpu").pin_memory(), dl.lse))
+        d2h_pairs.append((torch.empty_like(dl.idx, device="cpu").pin_memory(), dl.idx))
+    for src in dc._append_src:
+        h2d_pairs.append((src.cpu().pin_memory(), src))
+    bi = sum(h.numel() * h.element_size() for h, _ in h2d_pairs)
+    bo = sum(h.numel() * h.element_size() for h, _ in d2h_pairs)
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        for h, d in h2d_pairs:
+            d.copy_(h, non_blocking=True)
+        step()
+        for h, d in d2h_pairs:
+            h.copy_(d, non_blocking=True)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    if rank != 0:
+        return
+    hbm_peak, _, peak_kind = _peaks()
+    tokens = cfg.B * world
+    value = tokens / (ms_max * 1e-3)
+    alg = _algorithmic_bytes(cfg)
+    # dominant kernel: the Full layer's indexer scoring over all T positions
+    name = "index_score_decode[full]"
+    nl, tot = kernels.get(name, (0, 0.0))
+    per_launch_ms = tot / nl if nl else float("nan")
+    k_bytes = cfg.B * cfg.T * 64
+    achieved = k_bytes / (per_launch_ms * 1e-3) / 1e9 if nl else None
+    src = os.path.join(ROOT, "indexer_selected_sparse_csa2_b200", "csrc", "index_decode.cu")
+    traffic = _traffic_record(src)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8/fp4 storage, fp32 scores, fp16 MMA",
+        "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "B_per_gpu": cfg.B, "T": cfg.T, "H": cfg.H, "H_I": cfg.H_I,
+                   "K": cfg.K, "W": cfg.W, "layers": "Full+pool(2048x8), 3x Reindex-in-pool",
+                   "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
+        "step_hbm_gbs": round(alg / (ms_max * 1e-3) / 1e9, 1),
+        "step_hbm_frac": round(alg / (ms_max * 1e-3) / 1e9 / hbm_peak, 4),
+        "step_algorithmic_bytes": alg,
+        "roofline": {
+            "kernel": name,
+            "bound": "hbm",
+            "achieved": round(achieved, 1) if achieved else None,
+            "peak": hbm_peak,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm_peak, 4) if achieved else None,
+            "traffic": traffic,
+            "bytes_per_launch": k_bytes,
+            "launch_ms": round(per_launch_ms, 5),
+            "peak_kind": peak_kind,
+        },
+        "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / args.steps, 5)} for k, v in kernels.items()},
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4)},
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, seconds_budget=args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=30.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from csa_synth import get_config
+    cfg = get_config(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_gpu(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

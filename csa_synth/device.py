@@ -1,0 +1,149 @@
+"""Device-resident workloads for the CUDA path (GPU tests and the benchmark).
+
+The fp32 / bf16 values come from ``csa_synth.workload`` (seeded, chunked);
+they are uploaded and encoded ON THE DEVICE by the library under test
+(``csa_quant_kv``), exactly as a caller would fill its caches.  The oracle
+never imports this module: it encodes the same values with its own code.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional
+
+import numpy as np
+
+from . import workload as wl
+from .configs import Config, FULL, REINDEX, REUSE
+
+UPLOAD_ROWS = 1 << 16
+
+
+def _lib():
+    import indexer_selected_sparse_csa2_b200 as csa
+    return csa
+
+
+@dataclass
+class DeviceLayer:
+    qI: object                      # uint8 [B, n_q, H_I, 64]
+    w: object                       # fp32 [B, n_q, H_I]
+    q: object                       # fp32 [B, n_q, H, 512]
+    win: object                     # uint8 [B, win_rows, 528]
+    idx: object                     # int32 [B, n_q, K]
+    out: object                     # fp32 [B, n_q, H, 512]
+    lse: object                     # fp32 [B, n_q, H]
+    sink: Optional[object] = None
+    pool: Optional[object] = None   # int32 [B, pool_blocks * pool_block_len]
+    pool_len: Optional[object] = None
+    scores: Optional[object] = None
+
+
+class DeviceCase:
+    """All caches and per-layer tensors of one config on ``device``."""
+
+    def __init__(self, cfg: Config, device: str = "cuda", sinks: bool = False, threads: int = 8,
+                 keep_scores: bool = False, batches: Optional[List[int]] = None):
+        import torch
+        csa = _lib()
+        self.cfg = cfg
+        self.device = device
+        B, T = cfg.B, cfg.T
+        self.keys: Dict[int, object] = {}
+        self.kv: Dict[int, object] = {}
+        for o in cfg.owners:
+            keys = torch.empty((B, T, cfg.d_I), dtype=torch.uint8, device=device)
+            kv = torch.empty((B, T, csa.FP4_ENTRY_BYTES), dtype=torch.uint8, device=device)
+            for b in range(B):
+                for t0 in range(0, T, UPLOAD_ROWS):
+                    n = min(UPLOAD_ROWS, T - t0)
+                    kx = torch.from_numpy(wl.index_key(cfg, o, b, t0, n, threads=threads)).to(device)
+                    csa.csa_quant_kv(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, t0:t0 + n])
+                    mx = self._latent_tensor(wl.main_latent(cfg, o, b, t0, n, threads=threads))
+                    csa.csa_quant_kv(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, t0:t0 + n])
+            self.keys[o] = keys
+            self.kv[o] = kv
+        self.layers: List[DeviceLayer] = []
+        for li, L in enumerate(cfg.layers):
+            qI_f = np.stack([wl.index_query(cfg, li, b) for b in range(B)])         # [B, n_q, H_I, 64]
+            qI = torch.empty(qI_f.shape, dtype=torch.uint8, device=device)
+            qf = torch.from_numpy(qI_f.reshape(-1, cfg.d_I)).to(device)
+            csa.csa_quant_kv(qf, csa.CSA_FMT_FP8_E4M3_PLAIN, qI.view(-1, cfg.d_I))
+            w = torch.from_numpy(np.stack([wl.index_weight(cfg, li, b) for b in range(B)])).to(device)
+            q = torch.from_numpy(np.stack([wl.attn_query(cfg, li, b) for b in range(B)])).to(device)
+            win = torch.empty((B, cfg.win_rows, csa.FP8_ENTRY_BYTES), dtype=torch.uint8, device=device)
+            for b in range(B):
+                wx = self._latent_tensor(wl.window_latent(cfg, li, b))
+                csa.csa_quant_kv(wx, csa.CSA_FMT_FP8_E4M3_UE8M0X32, win[b])
+            dl = DeviceLayer(
+                qI=qI, w=w.contiguous(), q=q.contiguous(), win=win,
+                idx=torch.full((B, cfg.n_q, cfg.K), -7, dtype=torch.int32, device=device),
+                out=torch.zeros((B, cfg.n_q, cfg.H, cfg.D), dtype=torch.float32, device=device),
+                lse=torch.zeros((B, cfg.n_q, cfg.H), dtype=torch.float32, device=device),
+            )
+            if sinks:
+                dl.sink = torch.from_numpy(wl.sink(cfg, li)).to(device)
+            if L.build_pool:
+                dl.pool = torch.full((B, cfg.pool_blocks * cfg.pool_block_len), -7, dtype=torch.int32,
+                                     device=device)
+                dl.pool_len = torch.zeros(B, dtype=torch.int32, device=device)
+            if keep_scores and L.mode != REUSE:
+                n = cfg.T
+                if L.mode == REINDEX and L.pool_from >= 0:
+                    n = cfg.pool_blocks * cfg.pool_block_len
+                dl.scores = torch.zeros((B, n), dtype=torch.float32, device=device)
+            self.layers.append(dl)
+
+    def _latent_tensor(self, x: np.ndarray):
+        import torch
+        t = torch.from_numpy(x).to(self.device)
+        return t.to(torch.bfloat16) if self.cfg.bf16_latents else t
+
+    # ------------------------------------------------------------------
+    def layer_descs(self, append_rows: bool = False):
+        """ctypes LayerDesc array for the config's stack.  With ``append_rows``
+        every owner layer re-encodes the newest token (position T-1) of its
+        main KV and indexer key, and every layer its newest window row, as part
+        of the step (values from the seeded generator)."""
+        import torch
+        csa = _lib()
+        cfg = self.cfg
+        descs = []
+        self._append_src = []
+        for li, L in enumerate(cfg.layers):
+            d = csa.LayerDesc()
+            d.mode = L.mode
+            d.reuse_from = L.reuse_from
+            d.pool_from = L.pool_from
+            dl = self.layers[li]
+            o = L.owner
+            if append_rows:
+                jobs = []
+                if o == li:
+                    mx = torch.stack([self._latent_tensor(wl.main_latent(cfg, o, b, cfg.T - 1, 1))[0]
+                                      for b in range(cfg.B)])
+                    kx = torch.from_numpy(np.stack([wl.index_key(cfg, o, b, cfg.T - 1, 1)[0]
+                                                    for b in range(cfg.B)])).to(self.device)
+                    kvrow = self.kv[o][:, cfg.T - 1]
+                    krow = self.keys[o][:, cfg.T - 1]
+                    jobs.append(csa.quant_job(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kvrow,
+                                              self.kv[o].stride(0)))
+                    jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, self.keys[o].stride(0)))
+                    self._append_src += [mx, kx]
+                wx = torch.stack([self._latent_tensor(wl.window_latent(cfg, li, b))[cfg.win_rows - 1]
+                                  for b in range(cfg.B)])
+                wrow = dl.win[:, cfg.win_rows - 1]
+                jobs.append(csa.quant_job(wx, csa.CSA_FMT_FP8_E4M3_UE8M0X32, wrow, dl.win.stride(0)))
+                self._append_src.append(wx)
+                for k, j in enumerate(jobs):
+                    d.append[k] = j
+            if L.mode != REUSE:
+                d.index = csa.index_args(
+                    keys=self.keys[o], q=dl.qI, w=dl.w, K=cfg.K, idx=dl.idx, T=cfg.T, n_q=cfg.n_q,
+                    pool_out=dl.pool, pool_out_len=dl.pool_len, pool_blocks=cfg.pool_blocks,
+                    pool_block_len=cfg.pool_block_len, scores=dl.scores)
+            d.attn = csa.attn_args(q=dl.q, kv=self.kv[o], idx=None, win=dl.win, n_win=cfg.n_win,
+                                   softmax_scale=cfg.softmax_scale, out=dl.out, lse=dl.lse, sink=dl.sink,
+                                   K=0)
+            descs.append(d)
+        return csa.make_layer_array(descs)

@@ -1,0 +1,239 @@
+/*
+ * csa.h - C ABI of the CSA2 compressed sparse-attention step (sm_100a).
+ *
+ * The step, per decode (or prefill) token of one attention layer:
+ *   (a) encode main-KV latents as FP4 E2M1 with one E4M3 scale per 16
+ *       channels (288-byte entries), the sliding-window KV as FP8 E4M3 with
+ *       one UE8M0 scale per 32 channels (528-byte entries), and indexer keys /
+ *       queries as plain E4M3;
+ *   (b) score every cached position (or a candidate pool) with the lightning
+ *       indexer S[s] = sum_j w[j] * relu(<qI[j], kI[s]>) and keep the Top-K;
+ *   (c) MLA attention of the query heads over the selected FP4 entries plus
+ *       the FP8 window (keys = values = the 512-wide dequantised latent).
+ * Layers run in one of three modes: Full, Reindex, Reuse.
+ *
+ * Sources: DeepSeek-V4.1 blog, "DeepSeek-V4.1-Flash" section, CSA2 paragraph
+ * (modes, hierarchical indexer, FP4 main KV with E4M3 per 16 channels);
+ * DeepSeek-V4.1-Flash architecture database (cache owners and sharing, entry
+ * storage formats, "2048-block x 8-position candidate pool");
+ * Model techniques map - DeepSeek-V4.1-Flash ("Indexer-selected sparse
+ * attention", "Sliding-window attention", "Learnable attention sink",
+ * "Multi-head latent attention" rows).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates, frees or synchronises; work is enqueued on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Transient memory is the caller's `workspace`, sized by the matching
+ *     *_workspace_size() call (0 bytes is valid when the size is 0).
+ *   - Arguments are checked on the host before any launch; a failed check
+ *     returns a non-zero csa_status and enqueues nothing.  A failed launch
+ *     returns CSA_ERR_CUDA.
+ *   - Byte strides and entry pointers must be 16-byte aligned.
+ *   - Calls keep no state between them and may be captured in a CUDA graph.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa_stream_t;
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1, /* NULL where a pointer is required, unknown enum */
+  CSA_ERR_SHAPE = 2,       /* a size outside the supported range */
+  CSA_ERR_ALIGNMENT = 3,   /* pointer or stride not 16-byte aligned */
+  CSA_ERR_UNSUPPORTED = 4, /* valid combination that is not implemented */
+  CSA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than required */
+  CSA_ERR_CUDA = 6         /* a kernel launch failed */
+} csa_status;
+
+typedef enum { CSA_SRC_F32 = 0, CSA_SRC_BF16 = 1 } csa_src_dtype;
+
+typedef enum {
+  /* 512 channels -> 288 B: bytes 0..255 = E2M1 codes, two per byte, even
+   * channel in the low nibble; bytes 256..287 = E4M3 scale of each block of
+   * 16 channels.  scale = E4M3_rne_sat(amax/6); code = E2M1_rne_sat(x/scale)
+   * (fp32 IEEE divisions); a zero scale gives all codes +0. */
+  CSA_FMT_FP4_E2M1_E4M3X16 = 0,
+  /* 512 channels -> 528 B: bytes 0..511 = E4M3 codes; bytes 512..527 = UE8M0
+   * exponent byte (e + 127) of each block of 32 channels, where e is the
+   * smallest integer with amax <= 448 * 2^e, clamped to [-127, 127];
+   * code = E4M3_rne_sat(x * 2^-e). */
+  CSA_FMT_FP8_E4M3_UE8M0X32 = 1,
+  /* dim channels -> dim bytes of E4M3_rne_sat(x) (indexer keys/queries). */
+  CSA_FMT_FP8_E4M3_PLAIN = 2
+} csa_kv_format;
+
+typedef enum { CSA_MODE_FULL = 0, CSA_MODE_REINDEX = 1, CSA_MODE_REUSE = 2 } csa_mode;
+
+/* ------------------------------------------------------------------------ */
+/* (a) Encode rows.
+ *   src            : n_rows rows of `dim` fp32 or bf16 values, row r at
+ *                    src + r * src_row_stride elements.
+ *   dim            : 512 for the FP4 / windowed FP8 formats; a positive
+ *                    multiple of 16 for CSA_FMT_FP8_E4M3_PLAIN.
+ *   dst            : row r written at dst + r * dst_row_stride bytes
+ *                    (288, 528 or dim bytes per row).
+ * Encodings are bit-exact functions of the inputs (round to nearest even,
+ * saturating); see csa_kv_format.  Non-finite inputs are outside the
+ * contract. */
+csa_status csa_quant_kv(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim,
+                        int64_t src_row_stride, int32_t fmt, void* dst,
+                        int64_t dst_row_stride, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* (b) Lightning-indexer scores + Top-K (optionally building or searching the
+ * hierarchical candidate pool).
+ *
+ * Query t (0 <= t < n_q) of sequence b sits at position T - n_q + t and
+ * scores positions [0, T - n_q + t]  (decode: n_q = 1, all of [0, T)).
+ *   S[s] = sum_j w[b,t,j] * max(0, sum_d qI[b,t,j,d] * kI[b,s,d])
+ * Top-K keeps the K largest S, ties broken towards the lower position, and
+ * writes the positions ASCENDING to idx[b,t,0..K), padding with -1 when fewer
+ * than K candidates exist.
+ *
+ * Pool search (pool != NULL, decode only): the candidates of sequence b are
+ * the positions pool[b, 0..pool_len[b]) (ascending, as written by pool_out).
+ * Pool build (pool_out != NULL, decode only): positions are grouped in
+ * aligned blocks of pool_block_len; a block scores the max of its positions;
+ * the pool_blocks best blocks (ties -> lower block) give pool_out[b] =
+ * their positions ascending (-1 padded to pool_blocks*pool_block_len) and
+ * pool_out_len[b] = the number of valid positions.
+ */
+typedef struct {
+  int32_t B;                 /* sequences, >= 1 */
+  int32_t n_q;               /* query tokens per sequence, >= 1 */
+  int64_t T;                 /* cache length, n_q <= T < 2^31 (n_q > 1:
+                                CSA_ERR_UNSUPPORTED in this version) */
+  int32_t H_I;               /* indexer heads, 1..8 */
+  int32_t d_I;               /* indexer head dim; must be 64 */
+  const uint8_t* keys;       /* E4M3 key of position s of sequence b at
+                                keys + b*key_batch_stride + s*key_row_stride */
+  int64_t key_row_stride;    /* bytes, >= 64, multiple of 16 */
+  int64_t key_batch_stride;  /* bytes, multiple of 16 */
+  const uint8_t* q;          /* E4M3 [B][n_q][H_I][64], contiguous */
+  const float* w;            /* fp32 [B][n_q][H_I], contiguous */
+  int32_t K;                 /* 1..65536 */
+  const int32_t* pool;       /* optional [B][pool_cap] ascending positions */
+  const int32_t* pool_len;   /* [B] valid entries of pool (required with pool) */
+  int32_t pool_cap;          /* row length of pool */
+  int32_t* pool_out;         /* optional [B][pool_blocks*pool_block_len] */
+  int32_t* pool_out_len;     /* [B] (required with pool_out) */
+  int32_t pool_blocks;       /* blocks kept in the pool, 1..65536 */
+  int32_t pool_block_len;    /* positions per block: 1, 2, 4, 8 or 16 */
+  int32_t* idx;              /* out: int32 [B][n_q][K] */
+  float* scores;             /* optional out (decode only): fp32 scores
+                                [B][T] (or [B][pool_cap] when searching a
+                                pool; slots past pool_len are not written) */
+} csa_index_args;
+
+size_t csa_index_workspace_size(const csa_index_args* a);
+csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t workspace_bytes,
+                          csa_stream_t stream);
+
+/* Top-K of given fp32 scores (same selection rule as csa_index_topk):
+ * row b is scores + b*row_stride (elements), n values; idx is [B][K]. */
+size_t csa_topk_workspace_size(int32_t B, int64_t n);
+csa_status csa_topk_scores(const float* scores, int32_t B, int64_t n, int64_t row_stride,
+                           int32_t K, int32_t* idx, void* workspace, size_t workspace_bytes,
+                           csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* (c) Sparse MLA attention.  For query t of sequence b and head h:
+ *   entries = { dequant(kv entry idx[b,t,i]) : idx >= 0 }  followed by
+ *             { dequant(window row t + r) : 0 <= r < n_win }   (duplicates kept)
+ *   l_e  = softmax_scale * <q[b,t,h], x_e>
+ *   out  = sum_e softmax(l, sink_h)_e * x_e ;  lse = log(sum_e exp(l_e) [+ exp(sink_h)])
+ * x_e is all 512 latent channels (keys = values).  The window rows of
+ * sequence b are at win + b*win_batch_stride + r*win_row_stride (528-B
+ * entries); main entries at kv + b*kv_batch_stride + s*kv_row_stride (288 B).
+ * Window entries are computed in fp16 and must decode to |x| < 65504. */
+typedef struct {
+  int32_t B, n_q, H, D;      /* H in {16, 32, 64}; D must be 512 */
+  const float* q;            /* fp32 [B][n_q][H][D] */
+  const uint8_t* kv;         /* FP4 main-KV entries */
+  int64_t kv_row_stride;     /* bytes, >= 288, multiple of 16 */
+  int64_t kv_batch_stride;   /* bytes, multiple of 16 */
+  const int32_t* idx;        /* int32 [B][n_q][K], -1 = no entry */
+  int32_t K;                 /* 0..65536 */
+  const uint8_t* win;        /* FP8 window entries (may be NULL when n_win = 0) */
+  int64_t win_row_stride;    /* bytes, >= 528, multiple of 16 */
+  int64_t win_batch_stride;  /* bytes, multiple of 16 */
+  int32_t n_win;             /* window entries per query, 0..1024 */
+  float softmax_scale;
+  const float* sink;         /* optional fp32 [H] sink logits */
+  float* out;                /* fp32 [B][n_q][H][D] */
+  float* lse;                /* optional fp32 [B][n_q][H] (natural log) */
+} csa_attn_args;
+
+size_t csa_attn_workspace_size(const csa_attn_args* a);
+csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t workspace_bytes,
+                           csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* A stack of layers run in order on one stream.
+ *   FULL    : encode `append` rows, index.* scoring + Top-K (+ pool build),
+ *             then attention with attn.idx = index.idx.
+ *   REINDEX : as FULL (index.keys and attn.kv normally point at the owner
+ *             layer's caches); with pool_from >= 0, index.pool / pool_len /
+ *             pool_cap are taken from layer pool_from's pool_out.
+ *   REUSE   : no scoring; attention with attn.idx = the idx of layer
+ *             reuse_from (attn.K likewise).
+ * `append[i]` with src != NULL encodes new rows (e.g. this step's token)
+ * into the caches before the layer's scoring. */
+typedef struct {
+  const void* src;           /* NULL = no job */
+  int32_t src_dtype;
+  int32_t dim;
+  int64_t n_rows;
+  int64_t src_row_stride;    /* elements */
+  int32_t fmt;
+  void* dst;
+  int64_t dst_row_stride;    /* bytes */
+} csa_quant_job;
+
+typedef struct {
+  int32_t mode;              /* csa_mode */
+  int32_t reuse_from;        /* REUSE: earlier layer index */
+  int32_t pool_from;         /* REINDEX: earlier layer that built a pool, or -1 */
+  csa_quant_job append[3];
+  csa_index_args index;      /* unused for REUSE */
+  csa_attn_args attn;        /* attn.idx / attn.K are filled in by the step */
+} csa_layer_desc;
+
+size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers);
+csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
+                          size_t workspace_bytes, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Opt-in timing of the library's own kernels (profiling support, no
+ * counterpart on the pages).  While enabled, each kernel launch is bracketed
+ * by two CUDA events recorded on its launch stream.  csa_profile_collect()
+ * waits for the recorded events, writes up to max_entries per-kernel totals
+ * (name, launches, summed milliseconds) and forgets them; it returns the
+ * number of distinct kernel names seen. */
+typedef struct {
+  char name[56];
+  uint64_t launches;
+  double total_ms;
+} csa_kernel_time;
+int32_t csa_profile_enable(int32_t on);   /* returns the previous state */
+int32_t csa_profile_collect(csa_kernel_time* out, int32_t max_entries);
+
+/* ------------------------------------------------------------------------ */
+const char* csa_status_string(int32_t status);
+/* Number of kernels the library has enqueued since load (all entry points). */
+uint64_t csa_launch_count(void);
+int32_t csa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H_ */

@@ -1,0 +1,289 @@
+// C ABI of the CSA2 sparse-attention step: argument checks, workspace
+// layout, dispatch, and the Full / Reindex / Reuse layer stack.
+//
+// Layer modes follow the DeepSeek-V4.1 blog ("DeepSeek-V4.1-Flash" section,
+// CSA2 paragraph: each attention layer is statically Full, Reindex or Reuse;
+// main KV and indexer K are shared across layers and Top-K indices reused;
+// the decoder's first Full layer builds the candidate pool later indexers
+// search) and the DeepSeek-V4.1-Flash architecture database (cache-sharing
+// fact: caches owned by source layers, read by the others; every layer keeps
+// its own 128-token window).
+#include <algorithm>
+#include <atomic>
+
+#include "select.cuh"
+
+namespace csa {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
+                         int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream);
+size_t index_decode_ws_bytes(const csa_index_args* a);
+cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream);
+size_t attn_ws_bytes(const csa_attn_args* a);
+cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream);
+
+static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+static bool al16i(int64_t v) { return (v & 15) == 0; }
+
+static csa_status check_quant(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim,
+                              int64_t src_row_stride, int32_t fmt, const void* dst, int64_t dst_row_stride) {
+  if (src_dtype != CSA_SRC_F32 && src_dtype != CSA_SRC_BF16) return CSA_ERR_INVALID_ARG;
+  if (fmt != CSA_FMT_FP4_E2M1_E4M3X16 && fmt != CSA_FMT_FP8_E4M3_UE8M0X32 && fmt != CSA_FMT_FP8_E4M3_PLAIN)
+    return CSA_ERR_INVALID_ARG;
+  if (n_rows < 0) return CSA_ERR_SHAPE;
+  if (n_rows == 0) return CSA_OK;
+  if (!src || !dst) return CSA_ERR_INVALID_ARG;
+  if (fmt == CSA_FMT_FP8_E4M3_PLAIN) {
+    if (dim <= 0 || dim % 16) return CSA_ERR_SHAPE;
+  } else if (dim != kD) {
+    return CSA_ERR_SHAPE;
+  }
+  const int64_t esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  if (src_row_stride < dim) return CSA_ERR_SHAPE;
+  const int64_t row_bytes = fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? kFp4Bytes : (fmt == CSA_FMT_FP8_E4M3_UE8M0X32 ? kFp8Bytes : dim);
+  if (n_rows > 1 && dst_row_stride < row_bytes) return CSA_ERR_SHAPE;
+  if (!al16(src) || !al16i(src_row_stride * esz) || !al16(dst) || !al16i(dst_row_stride)) return CSA_ERR_ALIGNMENT;
+  return CSA_OK;
+}
+
+static csa_status check_index(const csa_index_args* a) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 1 || a->n_q < 1 || a->T < a->n_q || a->T >= ((int64_t)1 << 31)) return CSA_ERR_SHAPE;
+  if (a->H_I < 1 || a->H_I > 8 || a->d_I != kDI) return CSA_ERR_SHAPE;
+  if (a->K < 1 || a->K > 65536) return CSA_ERR_SHAPE;
+  if (!a->keys || !a->q || !a->w || !a->idx) return CSA_ERR_INVALID_ARG;
+  if (a->key_row_stride < kDI) return CSA_ERR_SHAPE;
+  if (!al16(a->keys) || !al16i(a->key_row_stride) || !al16i(a->key_batch_stride) || !al16(a->q))
+    return CSA_ERR_ALIGNMENT;
+  if (a->n_q > 1) {
+    if (a->pool || a->pool_out || a->scores) return CSA_ERR_UNSUPPORTED;
+    return CSA_ERR_UNSUPPORTED;   // prefill scoring is provided by the GEMM path
+  }
+  if (a->pool && a->pool_out) return CSA_ERR_UNSUPPORTED;
+  if (a->pool) {
+    if (!a->pool_len || a->pool_cap < 1) return CSA_ERR_INVALID_ARG;
+  }
+  if (a->pool_out) {
+    if (!a->pool_out_len) return CSA_ERR_INVALID_ARG;
+    const int bl = a->pool_block_len;
+    if (a->pool_blocks < 1 || a->pool_blocks > 65536) return CSA_ERR_SHAPE;
+    if (bl != 1 && bl != 2 && bl != 4 && bl != 8 && bl != 16) return CSA_ERR_SHAPE;
+  }
+  return CSA_OK;
+}
+
+static csa_status check_attn(const csa_attn_args* a) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 1 || a->n_q < 1) return CSA_ERR_SHAPE;
+  if (a->H != 16 && a->H != 32 && a->H != 64) return CSA_ERR_SHAPE;
+  if (a->D != kD) return CSA_ERR_SHAPE;
+  if (a->K < 0 || a->K > 65536 || a->n_win < 0 || a->n_win > 1024) return CSA_ERR_SHAPE;
+  if (!a->q || !a->out) return CSA_ERR_INVALID_ARG;
+  if (a->K > 0 && (!a->kv || !a->idx)) return CSA_ERR_INVALID_ARG;
+  if (a->n_win > 0 && !a->win) return CSA_ERR_INVALID_ARG;
+  if (a->K > 0 && (a->kv_row_stride < kFp4Bytes || !al16(a->kv) || !al16i(a->kv_row_stride) ||
+                   !al16i(a->kv_batch_stride)))
+    return a->kv_row_stride < kFp4Bytes ? CSA_ERR_SHAPE : CSA_ERR_ALIGNMENT;
+  if (a->n_win > 0 && (a->win_row_stride < kFp8Bytes || !al16(a->win) || !al16i(a->win_row_stride) ||
+                       !al16i(a->win_batch_stride)))
+    return a->win_row_stride < kFp8Bytes ? CSA_ERR_SHAPE : CSA_ERR_ALIGNMENT;
+  if (!al16(a->q) || !al16(a->out)) return CSA_ERR_ALIGNMENT;
+  return CSA_OK;
+}
+
+static csa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+csa_status csa_quant_kv(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim,
+                        int64_t src_row_stride, int32_t fmt, void* dst, int64_t dst_row_stride,
+                        csa_stream_t stream) {
+  csa_status s = check_quant(src, src_dtype, n_rows, dim, src_row_stride, fmt, dst, dst_row_stride);
+  if (s != CSA_OK || n_rows == 0) return s;
+  return from_cuda(launch_quant(src, src_dtype, n_rows, dim, src_row_stride, fmt, dst, dst_row_stride,
+                                (cudaStream_t)stream));
+}
+
+size_t csa_index_workspace_size(const csa_index_args* a) {
+  if (check_index(a) != CSA_OK) return 0;
+  return index_decode_ws_bytes(a);
+}
+
+csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t workspace_bytes,
+                          csa_stream_t stream) {
+  csa_status s = check_index(a);
+  if (s != CSA_OK) return s;
+  const size_t need = index_decode_ws_bytes(a);
+  if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
+  if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
+  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream));
+}
+
+size_t csa_topk_workspace_size(int32_t B, int64_t n) {
+  if (B < 1 || n < 1) return 0;
+  return select_workspace_bytes(B, n);
+}
+
+csa_status csa_topk_scores(const float* scores, int32_t B, int64_t n, int64_t row_stride, int32_t K,
+                           int32_t* idx, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
+  if (!scores || !idx) return CSA_ERR_INVALID_ARG;
+  if (B < 1 || n < 1 || n >= ((int64_t)1 << 31) || row_stride < n || K < 1 || K > 65536) return CSA_ERR_SHAPE;
+  const size_t need = select_workspace_bytes(B, n);
+  if (need > workspace_bytes || !workspace) return CSA_ERR_WORKSPACE;
+  if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  SelectJob j{};
+  select_carve(j, B, n, workspace);
+  j.vals = scores;
+  j.row_stride = row_stride;
+  j.n_row = nullptr;
+  j.K = K;
+  j.out = idx;
+  j.out_stride = K;
+  j.out_width = K;
+  j.map = nullptr;
+  j.expand = 0;
+  cudaError_t e = launch_zero(j.hist, (size_t)B * kHistBins * 4, st);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  return from_cuda(launch_select(&j, 1, B, true, st));
+}
+
+size_t csa_attn_workspace_size(const csa_attn_args* a) {
+  if (check_attn(a) != CSA_OK) return 0;
+  return attn_ws_bytes(a);
+}
+
+csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t workspace_bytes,
+                           csa_stream_t stream) {
+  csa_status s = check_attn(a);
+  if (s != CSA_OK) return s;
+  const size_t need = attn_ws_bytes(a);
+  if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
+  if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
+  return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream));
+}
+
+// Resolve one layer of a stack into concrete index / attention arguments.
+static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_args* ix, csa_attn_args* at) {
+  const csa_layer_desc& d = L[i];
+  *at = d.attn;
+  if (d.mode == CSA_MODE_REUSE) {
+    if (d.reuse_from < 0 || d.reuse_from >= i) return CSA_ERR_INVALID_ARG;
+    int32_t src = d.reuse_from;
+    while (L[src].mode == CSA_MODE_REUSE) {            // a chain of reuse resolves to its source
+      if (L[src].reuse_from < 0 || L[src].reuse_from >= src) return CSA_ERR_INVALID_ARG;
+      src = L[src].reuse_from;
+    }
+    if (L[src].index.n_q != at->n_q || L[src].index.B != at->B) return CSA_ERR_SHAPE;
+    at->idx = L[src].index.idx;
+    at->K = L[src].index.K;
+    return CSA_OK;
+  }
+  if (d.mode != CSA_MODE_FULL && d.mode != CSA_MODE_REINDEX) return CSA_ERR_INVALID_ARG;
+  *ix = d.index;
+  if (d.mode == CSA_MODE_REINDEX && d.pool_from >= 0) {
+    if (d.pool_from >= i || !L[d.pool_from].index.pool_out) return CSA_ERR_INVALID_ARG;
+    const csa_index_args& P = L[d.pool_from].index;
+    ix->pool = P.pool_out;
+    ix->pool_len = P.pool_out_len;
+    ix->pool_cap = P.pool_blocks * P.pool_block_len;
+    ix->pool_out = nullptr;
+    ix->pool_out_len = nullptr;
+  } else if (d.mode == CSA_MODE_REINDEX) {
+    ix->pool = nullptr;
+  }
+  if (d.mode == CSA_MODE_FULL) ix->pool = nullptr;
+  if (ix->n_q != at->n_q || ix->B != at->B) return CSA_ERR_SHAPE;
+  at->idx = ix->idx;
+  at->K = ix->K;
+  return CSA_OK;
+}
+
+size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) {
+  if (!layers || n_layers < 1) return 0;
+  size_t need = 0;
+  for (int32_t i = 0; i < n_layers; ++i) {
+    csa_index_args ix{};
+    csa_attn_args at{};
+    if (resolve_layer(layers, i, &ix, &at) != CSA_OK) return 0;
+    if (layers[i].mode != CSA_MODE_REUSE) {
+      if (check_index(&ix) != CSA_OK) return 0;
+      need = std::max(need, index_decode_ws_bytes(&ix));
+    }
+    if (check_attn(&at) != CSA_OK) return 0;
+    need = std::max(need, attn_ws_bytes(&at));
+  }
+  return need;
+}
+
+csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
+                          size_t workspace_bytes, csa_stream_t stream) {
+  if (!layers || n_layers < 1) return CSA_ERR_INVALID_ARG;
+  // validate everything before enqueuing anything
+  size_t need = 0;
+  for (int32_t i = 0; i < n_layers; ++i) {
+    csa_index_args ix{};
+    csa_attn_args at{};
+    csa_status s = resolve_layer(layers, i, &ix, &at);
+    if (s != CSA_OK) return s;
+    for (int k = 0; k < 3; ++k) {
+      const csa_quant_job& q = layers[i].append[k];
+      if (!q.src) continue;
+      s = check_quant(q.src, q.src_dtype, q.n_rows, q.dim, q.src_row_stride, q.fmt, q.dst, q.dst_row_stride);
+      if (s != CSA_OK) return s;
+    }
+    if (layers[i].mode != CSA_MODE_REUSE) {
+      s = check_index(&ix);
+      if (s != CSA_OK) return s;
+      need = std::max(need, index_decode_ws_bytes(&ix));
+    }
+    s = check_attn(&at);
+    if (s != CSA_OK) return s;
+    need = std::max(need, attn_ws_bytes(&at));
+  }
+  if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
+  if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int32_t i = 0; i < n_layers; ++i) {
+    csa_index_args ix{};
+    csa_attn_args at{};
+    resolve_layer(layers, i, &ix, &at);
+    for (int k = 0; k < 3; ++k) {
+      const csa_quant_job& q = layers[i].append[k];
+      if (!q.src || q.n_rows == 0) continue;
+      if (launch_quant(q.src, q.src_dtype, q.n_rows, q.dim, q.src_row_stride, q.fmt, q.dst, q.dst_row_stride,
+                       st) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    }
+    if (layers[i].mode != CSA_MODE_REUSE) {
+      if (run_index_decode(&ix, workspace, st) != cudaSuccess) return CSA_ERR_CUDA;
+    }
+    if (run_sparse_attn(&at, workspace, st) != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  return CSA_OK;
+}
+
+const char* csa_status_string(int32_t s) {
+  switch (s) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case CSA_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case CSA_ERR_UNSUPPORTED: return "unsupported combination";
+    case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA_ERR_CUDA: return "CUDA launch failed";
+    default: return "unknown status";
+  }
+}
+
+uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+int32_t csa_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,173 @@
+// Cache-entry encoders: FP4 main KV, FP8 windowed KV, plain E4M3 cast.
+//
+// FP4 main-KV entry (DeepSeek-V4.1 blog, "DeepSeek-V4.1-Flash" section, CSA2
+// paragraph: E2M1 with one E4M3 scale per 16 channels; DeepSeek-V4.1-Flash
+// architecture database, storage of the main-KV groups: 256 data bytes + 32
+// float8_e4m3 scale bytes).  FP8 window entry (same database, storage of the
+// "SWA window" group: E4M3 data with E8M0 scales per 32 channels, 512 + 16
+// bytes).  Scale rules: see csa_kv_format in csa.h.
+//
+// One warp encodes one 512-channel row; lane l owns channels [16l, 16l+16),
+// i.e. exactly one FP4 scale block, or half of one FP8 scale block.  Rows are
+// read with 128-bit loads and written with 64/128-bit stores.
+#include "common.cuh"
+
+namespace csa {
+
+template <int SRC>  // 0 = fp32, 1 = bf16
+CSA_DEV void load16(const void* row, int lane, float (&x)[16]) {
+  if (SRC == 0) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(row) + 16 * lane);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 v = ld_nc_v4(p + i);
+      x[4 * i + 0] = __uint_as_float(v.x);
+      x[4 * i + 1] = __uint_as_float(v.y);
+      x[4 * i + 2] = __uint_as_float(v.z);
+      x[4 * i + 3] = __uint_as_float(v.w);
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(row) + 16 * lane);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint4 v = ld_nc_v4(p + i);
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        x[8 * i + 2 * k + 0] = __uint_as_float(w[k] << 16);          // bf16 -> fp32 is exact
+        x[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+      }
+    }
+  }
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__ src, int64_t n_rows,
+                                                        int64_t src_stride_bytes,
+                                                        uint8_t* __restrict__ dst, int64_t dst_stride) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
+    float x[16];
+    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, x);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const uint32_t s_code = enc_e4m3x2(0.f, __fdiv_rn(amax, 6.0f)) & 0xFF;
+    const float s = dec_e4m3(s_code);
+    uint32_t packed[2] = {0u, 0u};
+    if (s != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // even channel in the low nibble
+        uint32_t b = enc_e2m1x2(__fdiv_rn(x[2 * i + 1], s), __fdiv_rn(x[2 * i], s));
+        packed[i >> 2] |= b << (8 * (i & 3));
+      }
+    }
+    uint8_t* out = dst + r * dst_stride;
+    *reinterpret_cast<uint2*>(out + 8 * lane) = make_uint2(packed[0], packed[1]);
+    out[256 + lane] = (uint8_t)s_code;
+  }
+}
+
+// Smallest e with amax <= 448 * 2^e, clamped to [-127, 127]; amax == 0 -> -127.
+// amax = (1 + m / 2^23) * 2^E for a normal fp32; 448 = 1.75 * 2^8, so the
+// answer is E - 8 when the significand is at most 1.75 and E - 7 otherwise.
+CSA_DEV int ue8m0_exponent(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int ef = (int)((u >> 23) & 0xFF);
+  if (ef == 0) return -127;  // zero or subnormal: far below 448 * 2^-127
+  const uint32_t m = u & 0x7FFFFFu;
+  int e = (ef - 127) - 8 + (m > 0x600000u ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^k as an fp32 value for k in [-127, 127] (2^-127 is subnormal).
+CSA_DEV float pow2f(int k) {
+  return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << 22);
+}
+
+template <int SRC>
+__global__ void __launch_bounds__(256) quant_fp8w_kernel(const void* __restrict__ src, int64_t n_rows,
+                                                         int64_t src_stride_bytes,
+                                                         uint8_t* __restrict__ dst, int64_t dst_stride) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
+    float x[16];
+    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, x);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 32-channel block = lane pair
+    const int e = ue8m0_exponent(amax);
+    const float sc = pow2f(-e);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo = enc_e4m3x2(x[4 * i + 1] * sc, x[4 * i + 0] * sc);
+      uint32_t hi = enc_e4m3x2(x[4 * i + 3] * sc, x[4 * i + 2] * sc);
+      w[i] = lo | (hi << 16);
+    }
+    uint8_t* out = dst + r * dst_stride;
+    *reinterpret_cast<uint4*>(out + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    if ((lane & 1) == 0) out[512 + (lane >> 1)] = (uint8_t)(e + 127);
+  }
+}
+
+// Plain E4M3 cast: each thread encodes 16 consecutive values of one row.
+template <int SRC>
+__global__ void __launch_bounds__(256) quant_plain_kernel(const void* __restrict__ src, int64_t n_rows,
+                                                          int dim, int64_t src_stride_bytes,
+                                                          uint8_t* __restrict__ dst, int64_t dst_stride) {
+  const int per_row = dim >> 4;
+  const int64_t total = n_rows * per_row;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = g / per_row;
+    const int c = (int)(g - r * per_row);
+    float x[16];
+    // reuse the 16-value loader with "lane" = column group
+    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, c, x);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo = enc_e4m3x2(x[4 * i + 1], x[4 * i + 0]);
+      uint32_t hi = enc_e4m3x2(x[4 * i + 3], x[4 * i + 2]);
+      w[i] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(dst + r * dst_stride + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+static int grid_for(int64_t work, int per_block) {
+  int64_t g = (work + per_block - 1) / per_block;
+  const int64_t cap = (int64_t)kNumSMs * 16;
+  return (int)(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
+                         int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const int esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  const int64_t sstride = src_row_stride * esz;
+  uint8_t* d = static_cast<uint8_t*>(dst);
+  ProfScope ps(stream, fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? "quant_fp4" : (fmt == CSA_FMT_FP8_E4M3_UE8M0X32 ? "quant_fp8w" : "quant_plain"));
+  if (fmt == CSA_FMT_FP4_E2M1_E4M3X16) {
+    const int g = grid_for(n_rows, 8);
+    if (src_dtype == CSA_SRC_F32) quant_fp4_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+    else quant_fp4_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+  } else if (fmt == CSA_FMT_FP8_E4M3_UE8M0X32) {
+    const int g = grid_for(n_rows, 8);
+    if (src_dtype == CSA_SRC_F32) quant_fp8w_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+    else quant_fp8w_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+  } else {
+    const int g = grid_for(n_rows * (dim / 16), 256);
+    if (src_dtype == CSA_SRC_F32) quant_plain_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, dim, sstride, d, dst_row_stride);
+    else quant_plain_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, dim, sstride, d, dst_row_stride);
+  }
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

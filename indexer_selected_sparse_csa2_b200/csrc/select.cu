@@ -1,0 +1,366 @@
+// Exact Top-K selection (lowest-position tie-break, ascending output).
+//
+// Selection rule of the lightning indexer (Model techniques map -
+// DeepSeek-V4.1-Flash, "Indexer-selected sparse attention" row: each query
+// attends only to the index_topk best-scored tokens).  Ties are broken
+// towards the lower position so the result is one well-defined set.
+//
+// Three stages over rows of fp32 values (order_key maps them to uint32 keys
+// that sort like the values):
+//   hist    - 4096-bin histogram of key >> 20 per row (usually fused into the
+//             producer of the values, e.g. the indexer scoring kernel);
+//   extract - many CTAs per row: find the bin b1 holding the K-th largest key,
+//             then copy every slot whose bin is >= b1 into that CTA's own
+//             region of a candidate buffer, in slot order, plus a count;
+//   final   - one CTA per row: concatenate the candidate runs (still in slot
+//             order), run an 8-bit radix select on the full 32-bit key to get
+//             the exact K-th key tau and how many slots equal to tau are
+//             needed, then emit the selected slots in slot order (so the
+//             output is ascending and the lowest equal slots win).
+#include "select.cuh"
+
+namespace csa {
+
+constexpr int kExtractThreads = 256;
+constexpr int kFinalThreads = 1024;
+constexpr int kFinalSmemCap = 12288;    // candidates staged in shared memory
+constexpr int kMaxChunks = 1024;
+
+struct SelectJobs {
+  SelectJob j[2];
+};
+
+SelectPlan plan_select(int B, int64_t n) {
+  SelectPlan p;
+  // ~2 waves of extract CTAs over all rows; at least 4096 slots per CTA; at
+  // most kMaxChunks runs per row so the final CTA can scan the run counts.
+  int64_t target = (int64_t)kNumSMs * 4 / (B > 0 ? B : 1);
+  if (target < 1) target = 1;
+  int64_t chunk = (n + target - 1) / target;
+  if (chunk < 4096) chunk = 4096;
+  int64_t minc = (n + kMaxChunks - 1) / kMaxChunks;
+  if (chunk < minc) chunk = minc;
+  chunk = (chunk + 255) / 256 * 256;
+  p.chunk = chunk;
+  p.nchunks = (int)((n + chunk - 1) / chunk);
+  if (p.nchunks < 1) p.nchunks = 1;
+  return p;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t select_workspace_bytes(int B, int64_t n) {
+  SelectPlan p = plan_select(B, n);
+  size_t s = 0;
+  s += align256((size_t)B * kHistBins * 4);
+  s += 4 * align256((size_t)B * (size_t)(n > 0 ? n : 1) * 4);
+  s += align256((size_t)B * p.nchunks * 4);
+  return s;
+}
+
+size_t select_carve(SelectJob& j, int B, int64_t n, void* ws) {
+  SelectPlan p = plan_select(B, n);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = 0;
+  const size_t nn = (size_t)(n > 0 ? n : 1);
+  j.hist = reinterpret_cast<uint32_t*>(base + off); off += align256((size_t)B * kHistBins * 4);
+  j.cand_key = reinterpret_cast<uint32_t*>(base + off); off += align256((size_t)B * nn * 4);
+  j.cand_pos = reinterpret_cast<int32_t*>(base + off); off += align256((size_t)B * nn * 4);
+  j.list_key = reinterpret_cast<uint32_t*>(base + off); off += align256((size_t)B * nn * 4);
+  j.list_pos = reinterpret_cast<int32_t*>(base + off); off += align256((size_t)B * nn * 4);
+  j.cnt = reinterpret_cast<int32_t*>(base + off); off += align256((size_t)B * p.nchunks * 4);
+  j.chunk = p.chunk;
+  j.nchunks = p.nchunks;
+  j.n = n;
+  return off;
+}
+
+// ------------------------------------------------------------------ zero --
+__global__ void zero_kernel(uint4* p, size_t n16) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    p[i] = make_uint4(0, 0, 0, 0);
+}
+
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t stream) {
+  size_t n16 = bytes / 16;
+  if (n16 == 0) return cudaSuccess;
+  int g = (int)((n16 + 255) / 256);
+  if (g > kNumSMs * 8) g = kNumSMs * 8;
+  ProfScope ps(stream, "zero");
+  zero_kernel<<<g, 256, 0, stream>>>(static_cast<uint4*>(p), n16);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ hist --
+__global__ void __launch_bounds__(256) select_hist_kernel(SelectJobs jobs) {
+  const SelectJob& J = jobs.j[blockIdx.z];
+  const int b = blockIdx.y;
+  const int c = blockIdx.x;
+  if (c >= J.nchunks) return;
+  __shared__ uint32_t h[kHistBins];
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int64_t nrow = J.n_row ? (int64_t)min((int64_t)J.n_row[b], J.n) : J.n;
+  const int64_t lo = (int64_t)c * J.chunk;
+  const int64_t hi = min(lo + J.chunk, nrow);
+  const float* v = J.vals + (int64_t)b * J.row_stride;
+  for (int64_t s = lo + threadIdx.x; s < hi; s += blockDim.x) atomicAdd(&h[order_key(v[s]) >> (32 - kHistBits)], 1u);
+  __syncthreads();
+  uint32_t* g = J.hist + (int64_t)b * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (h[i]) atomicAdd(&g[i], h[i]);
+}
+
+// -------------------------------------------------------------- block scan --
+// Inclusive scan over the block (blockDim.x multiple of 32, <= 1024).
+template <int NT>
+CSA_DEV uint32_t block_incl_scan(uint32_t v, uint32_t* warp_tot, uint32_t* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) warp_tot[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = lane < NT / 32 ? warp_tot[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t t = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += t;
+    }
+    if (lane < NT / 32) warp_tot[lane] = w;
+    if (lane == NT / 32 - 1) *total = w;
+  }
+  __syncthreads();
+  const uint32_t r = v + (wid > 0 ? warp_tot[wid - 1] : 0u);
+  __syncthreads();
+  return r;
+}
+
+// Find the first-level threshold bin: the largest bin beta with
+// sum_{bins >= beta} >= K (0 when the row holds fewer than K values).
+CSA_DEV int threshold_bin(const uint32_t* gh, int K, uint32_t* warp_tot, uint32_t* total, int* out_bin) {
+  // thread i covers bins [16*(255-i), 16*(255-i)+16): scanning threads in
+  // order walks the bins from the top down.
+  static_assert(kHistBins == 256 * 16, "layout");
+  const int i = threadIdx.x;
+  uint32_t loc[16];
+  uint32_t s = 0;
+  const int base = 16 * (255 - i);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) { loc[k] = gh[base + k]; s += loc[k]; }
+  if (i == 0) *out_bin = 0;
+  const uint32_t incl = block_incl_scan<256>(s, warp_tot, total);
+  const uint32_t excl = incl - s;
+  if (excl < (uint32_t)K && incl >= (uint32_t)K) {
+    uint32_t cum = excl;
+    for (int k = 15; k >= 0; --k) {
+      cum += loc[k];
+      if (cum >= (uint32_t)K) { *out_bin = base + k; break; }
+    }
+  }
+  __syncthreads();
+  return *out_bin;
+}
+
+__global__ void __launch_bounds__(kExtractThreads) select_extract_kernel(SelectJobs jobs) {
+  const SelectJob& J = jobs.j[blockIdx.z];
+  const int b = blockIdx.y;
+  const int c = blockIdx.x;
+  if (c >= J.nchunks) return;
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t total;
+  __shared__ int bin;
+  const int beta = threshold_bin(J.hist + (int64_t)b * kHistBins, J.K, warp_tot, &total, &bin);
+  const int64_t nrow = J.n_row ? (int64_t)min((int64_t)J.n_row[b], J.n) : J.n;
+  const int64_t lo = (int64_t)c * J.chunk;
+  const int64_t hi = min(lo + J.chunk, nrow);
+  const float* v = J.vals + (int64_t)b * J.row_stride;
+  uint32_t* ck = J.cand_key + (int64_t)b * J.n + lo;
+  int32_t* cp = J.cand_pos + (int64_t)b * J.n + lo;
+  uint32_t run = 0;
+  for (int64_t s0 = lo; s0 < hi; s0 += kExtractThreads) {
+    const int64_t s = s0 + threadIdx.x;
+    uint32_t key = 0;
+    uint32_t f = 0;
+    if (s < hi) {
+      key = order_key(v[s]);
+      f = (int)(key >> (32 - kHistBits)) >= beta;
+    }
+    const uint32_t incl = block_incl_scan<kExtractThreads>(f, warp_tot, &total);
+    if (f) {
+      ck[run + incl - 1] = key;
+      cp[run + incl - 1] = (int32_t)s;
+    }
+    run += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) J.cnt[(int64_t)b * J.nchunks + c] = (int32_t)run;
+}
+
+// ----------------------------------------------------------------- final --
+CSA_DEV void write_selected(const SelectJob& J, int b, uint32_t j, int32_t slot) {
+  int32_t* out = J.out + (int64_t)b * J.out_stride;
+  int32_t pos = J.map ? J.map[(int64_t)b * J.map_stride + slot] : slot;
+  if (J.expand == 0) {
+    out[j] = pos;
+  } else {
+    for (int r = 0; r < J.expand; ++r) {
+      int64_t p = (int64_t)pos * J.expand + r;
+      out[(int64_t)j * J.expand + r] = p < J.limit ? (int32_t)p : -1;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs jobs) {
+  const SelectJob& J = jobs.j[blockIdx.y];
+  const int b = blockIdx.x;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint32_t* skey = reinterpret_cast<uint32_t*>(smem);
+  int32_t* spos = reinterpret_cast<int32_t*>(smem + kFinalSmemCap * 4);
+  __shared__ uint32_t offs[kMaxChunks];
+  __shared__ uint32_t warp_tot[32];
+  __shared__ uint32_t total;
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_prefix, s_krem;
+
+  // 1. run offsets
+  const int tid = threadIdx.x;
+  uint32_t cnt = tid < J.nchunks ? (uint32_t)J.cnt[(int64_t)b * J.nchunks + tid] : 0u;
+  const uint32_t incl = block_incl_scan<kFinalThreads>(cnt, warp_tot, &total);
+  offs[tid] = incl - cnt;
+  const uint32_t m = total;
+  __syncthreads();
+
+  // 2. contiguous ordered list (shared memory when it fits)
+  const bool in_smem = m <= (uint32_t)kFinalSmemCap;
+  uint32_t* lk = in_smem ? skey : J.list_key + (int64_t)b * J.n;
+  int32_t* lp = in_smem ? spos : J.list_pos + (int64_t)b * J.n;
+  for (int c = 0; c < J.nchunks; ++c) {
+    const uint32_t n_c = (uint32_t)J.cnt[(int64_t)b * J.nchunks + c];
+    const uint32_t* src_k = J.cand_key + (int64_t)b * J.n + (int64_t)c * J.chunk;
+    const int32_t* src_p = J.cand_pos + (int64_t)b * J.n + (int64_t)c * J.chunk;
+    for (uint32_t i = tid; i < n_c; i += kFinalThreads) {
+      lk[offs[c] + i] = src_k[i];
+      lp[offs[c] + i] = src_p[i];
+    }
+  }
+  __syncthreads();
+
+  // 3. exact threshold by 4 passes of an 8-bit radix select
+  const uint32_t K = (uint32_t)J.K;
+  bool take_all = m <= K;
+  if (tid == 0) { s_prefix = 0; s_krem = K; }
+  __syncthreads();
+  if (!take_all) {
+    uint32_t mask = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += kFinalThreads) hist[i] = 0;
+      __syncthreads();
+      const uint32_t prefix = s_prefix;
+      for (uint32_t i = tid; i < m; i += kFinalThreads) {
+        const uint32_t k = lk[i];
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // lane l covers digits [255-8l-7, 255-8l], scanning from the top
+        uint32_t loc[8];
+        uint32_t s = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { loc[k] = hist[255 - 8 * tid - k]; s += loc[k]; }
+        uint32_t inc = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+          if (tid >= o) inc += t;
+        }
+        const uint32_t exc = inc - s;
+        const uint32_t krem = s_krem;
+        if (exc < krem && inc >= krem) {
+          uint32_t cum = exc;
+          for (int k = 0; k < 8; ++k) {
+            if (cum + loc[k] >= krem) {
+              const uint32_t d = 255u - 8u * tid - k;
+              s_prefix = prefix | (d << shift);
+              s_krem = krem - cum;
+              break;
+            }
+            cum += loc[k];
+          }
+        }
+      }
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+  }
+  const uint32_t tau = s_prefix;
+  const uint32_t need_eq = s_krem;   // slots equal to tau to take (lowest first)
+
+  // 4. ordered emission
+  uint32_t eq_base = 0, out_base = 0;
+  for (uint32_t i0 = 0; i0 < m; i0 += kFinalThreads) {
+    const uint32_t i = i0 + tid;
+    uint32_t k = 0;
+    bool valid = i < m;
+    if (valid) k = lk[i];
+    const uint32_t is_eq = (valid && !take_all && k == tau) ? 1u : 0u;
+    const uint32_t eq_incl = block_incl_scan<kFinalThreads>(is_eq, warp_tot, &total);
+    const uint32_t eq_tot = total;
+    const bool sel = valid && (take_all || k > tau || (is_eq && eq_base + eq_incl - 1 < need_eq));
+    const uint32_t s_incl = block_incl_scan<kFinalThreads>(sel ? 1u : 0u, warp_tot, &total);
+    const uint32_t s_tot = total;
+    if (sel) write_selected(J, b, out_base + s_incl - 1, lp[i]);
+    eq_base += eq_tot;
+    out_base += s_tot;
+    __syncthreads();
+  }
+  // 5. padding and valid length
+  const int32_t width = J.out_width;
+  int32_t* out = J.out + (int64_t)b * J.out_stride;
+  const int64_t written = (int64_t)out_base * (J.expand ? J.expand : 1);
+  for (int64_t j = written + tid; j < width; j += kFinalThreads) out[j] = -1;
+  __syncthreads();
+  if (J.expand && J.out_len && tid == 0) {
+    // only the highest selected block can reach past the limit
+    int64_t bad = 0;
+    for (int64_t j = written - J.expand; j < written; ++j)
+      if (j >= 0 && out[j] < 0) ++bad;
+    J.out_len[b] = (int32_t)(written - bad);
+  }
+}
+
+cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hist, cudaStream_t stream) {
+  SelectJobs js;
+  js.j[0] = jobs[0];
+  js.j[1] = njobs > 1 ? jobs[1] : jobs[0];
+  int maxc = 0;
+  for (int i = 0; i < njobs; ++i) maxc = jobs[i].nchunks > maxc ? jobs[i].nchunks : maxc;
+  dim3 g(maxc, B, njobs);
+  if (build_hist) {
+    ProfScope ps(stream, "select_hist");
+    select_hist_kernel<<<g, 256, 0, stream>>>(js);
+    note_launches(1);
+  }
+  {
+    ProfScope ps(stream, "select_extract");
+    select_extract_kernel<<<g, kExtractThreads, 0, stream>>>(js);
+  }
+  const size_t smem = (size_t)kFinalSmemCap * 8;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr_set = true;
+  }
+  {
+    ProfScope ps(stream, "select_final");
+    select_final_kernel<<<dim3(B, njobs), kFinalThreads, smem, stream>>>(js);
+  }
+  note_launches(2);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

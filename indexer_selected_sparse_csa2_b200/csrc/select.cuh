@@ -1,0 +1,51 @@
+// Exact Top-K selection over rows of fp32 values (declarations).
+#pragma once
+#include "common.cuh"
+
+namespace csa {
+
+// One selection problem over B rows: the K largest values of each row, ties
+// broken towards the lower slot, written as ascending positions.
+struct SelectJob {
+  const float* vals;        // [B][row_stride] values (slot s of row b)
+  int64_t row_stride;
+  int64_t n;                // slots per row (upper bound)
+  const int32_t* n_row;     // optional per-row slot count (<= n)
+  uint32_t* hist;           // [B][kHistBins] counts of order_key >> 20 (filled before extract)
+  int K;
+  // candidate buffers (workspace)
+  uint32_t* cand_key;       // [B][n]
+  int32_t* cand_pos;        // [B][n]
+  uint32_t* list_key;       // [B][n] ordered contiguous copy (used when the list exceeds smem)
+  int32_t* list_pos;        // [B][n]
+  int32_t* cnt;             // [B][nchunks]
+  int64_t chunk;            // slots per extract CTA
+  int nchunks;
+  // output
+  int32_t* out;             // [B][out_stride]
+  int64_t out_stride;
+  int32_t out_width;        // entries per output row (K, or K * expand)
+  const int32_t* map;       // optional slot -> position map [B][map_stride]
+  int64_t map_stride;
+  int expand;               // 0: write slots; >0: write `expand` positions per selected slot
+  int32_t* out_len;         // [B] valid positions written (expand mode)
+  int64_t limit;            // expand mode: positions >= limit are dropped
+};
+
+struct SelectPlan {
+  int64_t chunk;
+  int nchunks;
+};
+
+SelectPlan plan_select(int B, int64_t n);
+// Bytes of workspace one SelectJob needs (hist + candidate buffers + counts).
+size_t select_workspace_bytes(int B, int64_t n);
+// Carve a job's buffers from `ws` (aligned), returning bytes used.
+size_t select_carve(SelectJob& j, int B, int64_t n, void* ws);
+
+// Launch: [optional hist] -> extract -> final for up to two jobs sharing B.
+cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hist,
+                          cudaStream_t stream);
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t stream);
+
+}  // namespace csa

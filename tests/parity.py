@@ -1,0 +1,53 @@
+"""Comparison rules shared by the GPU parity tests.
+
+* Encodings and Top-K of given fp32 scores: bit-exact.
+* Indexer Top-K sets: equal, except that every position in the symmetric
+  difference must have an oracle score within REL_TIE * |S_K| of the oracle's
+  K-th largest score S_K (GPU scores carry fp32 rounding; the oracle's are
+  exact), and the GPU row must be ascending with -1 padding.
+* Attention outputs: |gpu - oracle| <= ATOL + RTOL * |oracle| per element
+  (fp32 outputs; the kernel computes in fp16 operands / fp32 accumulation).
+"""
+import numpy as np
+
+REL_TIE = 1e-4
+RTOL = 2e-3
+ATOL = 1e-3
+
+
+def check_row_format(row: np.ndarray):
+    v = row[row >= 0]
+    assert np.all(row[len(v):] == -1), "padding must be trailing -1"
+    assert np.all(np.diff(v) > 0), "positions must be strictly ascending"
+
+
+def topk_diff(gpu_row, ora_row, score_of):
+    """Return (n_diff, worst relative distance to S_K) and assert the rule."""
+    gpu_row = np.asarray(gpu_row)
+    ora_row = np.asarray(ora_row)
+    check_row_format(gpu_row)
+    g = set(gpu_row[gpu_row >= 0].tolist())
+    o = set(ora_row[ora_row >= 0].tolist())
+    assert len(g) == len(o), (len(g), len(o))
+    diff = g ^ o
+    if not diff:
+        return 0, 0.0
+    so = np.array([score_of(p) for p in o])
+    S_K = so.min()
+    worst = max(abs(score_of(p) - S_K) for p in diff) / max(abs(S_K), 1e-30)
+    assert worst <= REL_TIE, f"{len(diff)} differing positions, worst {worst:.3e} relative to S_K"
+    return len(diff), worst
+
+
+def assert_close(gpu, ora, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ora = np.asarray(ora, dtype=np.float64)
+    assert gpu.shape == ora.shape, (gpu.shape, ora.shape)
+    both_inf = np.isneginf(gpu) & np.isneginf(ora)
+    err = np.abs(gpu - ora)
+    bound = ATOL + RTOL * np.abs(ora)
+    bad = ~((err <= bound) | both_inf)
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(bad, err - bound, -np.inf)), bad.shape)
+        raise AssertionError(f"{what}: {bad.sum()} elements out of tolerance; worst at {i}: "
+                             f"gpu={gpu[i]!r} oracle={ora[i]!r}")

@@ -1,0 +1,99 @@
+"""GPU parity of whole layer stacks (csa_layer_step) vs the oracle.
+
+Small versions of every decode workload; the seeded inputs are encoded on the
+device by the library and independently by the oracle.
+"""
+import numpy as np
+import pytest
+
+from csa_synth import get_config
+from csa_synth.configs import FULL, REINDEX, REUSE
+from oracle.case import SynthCase
+from oracle import indexer as oi
+from oracle import quant as oq
+from tests.parity import topk_diff, assert_close, check_row_format
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def csa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import indexer_selected_sparse_csa2_b200 as m
+    return m
+
+
+def _check_stack(csa, cfg, append=False, sinks=False, batches=None):
+    from csa_synth.device import DeviceCase
+    dc = DeviceCase(cfg, sinks=sinks)
+    descs = dc.layer_descs(append_rows=append)
+    csa.csa_layer_step(descs)
+    torch.cuda.synchronize()
+    batches = range(cfg.B) if batches is None else batches
+    for b in batches:
+        case = SynthCase(cfg, b, sinks=sinks)
+        res = case.run(keep_scores=True)
+        # caches encoded on the device equal the oracle's encodings
+        for o in cfg.owners:
+            assert np.array_equal(dc.keys[o][b].cpu().numpy(), case.keys(o))
+            sample = np.unique(np.concatenate([np.arange(min(cfg.T, 64)), [cfg.T - 1]]))
+            assert np.array_equal(dc.kv[o][b, sample].cpu().numpy(), case.main_entries(o, sample))
+        for li, L in enumerate(cfg.layers):
+            dl = dc.layers[li]
+            r = res[li]
+            if L.mode == REUSE:
+                # no scoring: the step attends over the source layer's indices
+                assert np.array_equal(r.idx, res[L.reuse_from].idx)
+            else:
+                g_idx = dl.idx[b, 0].cpu().numpy()
+                check_row_format(g_idx)
+                if L.mode == REINDEX and L.pool_from >= 0:
+                    P = res[L.pool_from]
+                    ppos = P.pool[:P.pool_len].astype(np.int64)
+                    S_full = np.full(cfg.T, np.nan)
+                    S_full[ppos] = r.scores[0]
+                else:
+                    S_full = r.scores[0]
+                topk_diff(g_idx, r.idx[0], lambda p: S_full[p])
+                if L.build_pool:
+                    gp = dl.pool[b].cpu().numpy()
+                    gn = int(dl.pool_len[b])
+                    check_row_format(gp)
+                    bm = oi.block_max(r.scores[0], cfg.pool_block_len)
+                    gblk = np.unique(gp[:gn] // cfg.pool_block_len)
+                    oblk = np.unique(r.pool[:r.pool_len] // cfg.pool_block_len)
+                    pad = lambda a: np.concatenate([a, -np.ones(cfg.pool_blocks - a.size, np.int64)])
+                    topk_diff(pad(gblk), pad(oblk), lambda p: bm[p])
+            # attention: compare where the index sets agree exactly
+            src_layer = li if L.mode != REUSE else L.reuse_from
+            g_sel = dc.layers[src_layer].idx[b, 0].cpu().numpy()
+            if np.array_equal(g_sel, r.idx[0]):
+                assert_close(dl.out[b, 0].cpu().numpy(), r.out[0], f"layer {li} out")
+                assert_close(dl.lse[b, 0].cpu().numpy(), r.lse[0], f"layer {li} lse")
+
+
+def test_tiny_decode(csa):
+    _check_stack(csa, get_config("tiny_decode"))
+
+
+def test_tiny_decode_with_append_and_sinks(csa):
+    _check_stack(csa, get_config("tiny_decode"), append=True, sinks=True)
+
+
+def test_decode_outliers_small(csa):
+    _check_stack(csa, get_config("decode_64k", B=2, T=20000))
+
+
+def test_three_layer_stack_small(csa):
+    _check_stack(csa, get_config("stack_128k", B=3, T=9001))
+
+
+def test_hierarchical_small(csa):
+    _check_stack(csa, get_config("hier_1m", B=2, T=1 << 16))
+
+
+def test_hierarchical_ragged_tail(csa):
+    _check_stack(csa, get_config("hier_1m", B=1, T=20003, pool_blocks=700, K=300))
