@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m indexer_selected_sparse_csa2_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python indexer_selected_sparse_csa2_b200/build.py` "
         "(there is no CPU fallback)")
 
 _lib = ctypes.CDLL(LIB_PATH)

@@ -1,7 +1,8 @@
 """Build the CUDA library ``libcsa.so`` in-tree for sm_100a.
 
-Usage: ``python -m indexer_selected_sparse_csa2_b200.build`` (or ``build()``
-from ``__graft_entry__``).  Each ``csrc/*.cu`` is compiled to an object with
+Usage: ``python indexer_selected_sparse_csa2_b200/build.py [--force]`` (or
+``build()`` from ``__graft_entry__``); run it by path, since importing the
+package loads the library.  Each ``csrc/*.cu`` is compiled to an object with
 nvcc (``-gencode arch=compute_100a,code=sm_100a -lineinfo -O3``) and the
 objects are linked into one shared library next to this file.  Rebuilds only
 when a source or header is newer than the library.

@@ -366,51 +366,52 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
   }
 }
 
-// Merge the per-split partial results of one token (log-sum-exp combine).
-template <int H>
-__global__ void __launch_bounds__(256) attn_combine_kernel(AttnParams p) {
-  const int bt = blockIdx.x;
-  __shared__ float scale_s[H][17];   // per head: weight of each split (<= 16 splits cached)
-  __shared__ float inv_s[H];
+// Merge the per-split partial results (log-sum-exp combine): one CTA per
+// (token, head), 128 threads x 4 channels.
+__global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
+  const int bt = blockIdx.x, h = blockIdx.y, H = p.H;
   const int S = p.n_splits;
-  // per head: global max and denominator
-  for (int h = threadIdx.x; h < H; h += blockDim.x) {
-    float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, p.part_ml[(((int64_t)bt * S + s) * H + h) * 2]);
-    float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-    const float Mf = fmaxf(M, sk);
+  __shared__ float wgt_s[64];
+  __shared__ float inv_s, max_s;
+  const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
+  if (threadIdx.x < 32) {
+    float M = sk;
+    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, p.part_ml[(((int64_t)bt * S + s) * H + h) * 2]);
+    M = warp_max(M);
     float L = 0.f;
-    for (int s = 0; s < S; ++s) {
+    for (int s = threadIdx.x; s < S; s += 32) {
       const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (((int64_t)bt * S + s) * H + h) * 2);
-      const float wgt = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - Mf);
-      L += ml.y * wgt;
-      if (s < 16) scale_s[h][s] = wgt;
+      const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+      L += ml.y * w;
+      if (s < 64) wgt_s[s] = w;
     }
-    if (sk != -INFINITY) L += exp2f(sk - Mf);
-    inv_s[h] = L > 0.f ? 1.f / L : 0.f;
-    if (p.lse) p.lse[(int64_t)bt * H + h] = L > 0.f ? (Mf + log2f(L)) * kLn2 : -INFINITY;
-    scale_s[h][16] = Mf;
+    L = warp_sum(L);
+    if (threadIdx.x == 0) {
+      if (sk != -INFINITY) L += exp2f(sk - M);
+      inv_s = L > 0.f ? 1.f / L : 0.f;
+      if (p.lse) p.lse[(int64_t)bt * H + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+      max_s = M;
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < H * kD / 4; i += blockDim.x) {
-    const int h = (4 * i) / kD, d = (4 * i) % kD;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-      float wgt;
-      if (s < 16) {
-        wgt = scale_s[h][s];
-      } else {
-        const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
-        wgt = m == -INFINITY ? 0.f : exp2f(m - scale_s[h][16]);
-      }
-      if (wgt == 0.f) continue;
-      const float4 v = *reinterpret_cast<const float4*>(p.part_o + (((int64_t)bt * S + s) * H + h) * kD + d);
-      acc.x += wgt * v.x; acc.y += wgt * v.y; acc.z += wgt * v.z; acc.w += wgt * v.w;
+  const float M = max_s;
+  const int d = 4 * threadIdx.x;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < S; ++s) {
+    float w;
+    if (S <= 64) {
+      w = wgt_s[s];
+    } else {
+      const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
+      w = m == -INFINITY ? 0.f : exp2f(m - M);
     }
-    const float inv = inv_s[h];
-    *reinterpret_cast<float4*>(p.out + ((int64_t)bt * H + h) * kD + d) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (w == 0.f) continue;
+    const float4 v = *reinterpret_cast<const float4*>(p.part_o + (((int64_t)bt * S + s) * H + h) * kD + d);
+    acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
   }
+  const float inv = inv_s;
+  *reinterpret_cast<float4*>(p.out + ((int64_t)bt * H + h) * kD + d) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }
 
 template <int H>
@@ -430,6 +431,9 @@ static AttnPlan plan_attn(const csa_attn_args* a) {
   const int n_tiles = (n_entries + kTileE - 1) / kTileE;
   const int64_t tokens = (int64_t)a->B * a->n_q;
   int want = (int)((kNumSMs + tokens - 1) / tokens);
+  // at least two tiles per split: each split reloads q and writes a partial O
+  const int by_tiles = (n_tiles + 1) / 2;
+  if (want > by_tiles) want = by_tiles;
   if (want < 1) want = 1;
   if (want > n_tiles) want = n_tiles > 0 ? n_tiles : 1;
   pl.tiles_per_split = n_tiles > 0 ? (n_tiles + want - 1) / want : 1;
@@ -460,7 +464,7 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   note_launches(1);
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    attn_combine_kernel<H><<<p.B * p.n_q, 256, 0, stream>>>(p);
+    attn_combine_kernel<<<dim3(p.B * p.n_q, H), 128, 0, stream>>>(p);
     note_launches(1);
   }
   return cudaGetLastError();

@@ -22,8 +22,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def csa():
-    from indexer_selected_sparse_csa2_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import indexer_selected_sparse_csa2_b200 as m
     return m
 
