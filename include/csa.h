@@ -138,6 +138,25 @@ size_t csa_index_workspace_size(const csa_index_args* a);
 csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t workspace_bytes,
                           csa_stream_t stream);
 
+/* csa_index_topk without a workspace argument.  (The pages have no
+ * counterpart: this is a deployment variant of the call above.)
+ * For callers that cannot allocate device memory on their hot path (a
+ * runtime whose caching allocator already owns the GPU, or a loop that must
+ * not call cudaMalloc because it may synchronise the device): the scratch is
+ * a fixed 16 MiB array in the library's device image, held by every GPU that
+ * loads the library until the process exits.
+ *   - Same arguments and results as csa_index_topk.
+ *   - Returns CSA_ERR_WORKSPACE, before any launch, when
+ *     csa_index_workspace_size(a) > csa_index_noalloc_capacity().
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - Every call on a device shares the array, which keeps the last call's
+ *     contents (the kernels clear what must start at zero); calls that may
+ *     overlap on the GPU (unordered streams) race on it.
+ *   - Calls no cudaMalloc / cudaFree or allocating library routine. */
+size_t csa_index_noalloc_capacity(void);
+csa_status csa_index_topk_noalloc(const csa_index_args* a, csa_stream_t stream);
+
 /* Top-K of given fp32 scores (same selection rule as csa_index_topk):
  * row b is scores + b*row_stride (elements), n values; idx is [B][K]. */
 size_t csa_topk_workspace_size(int32_t B, int64_t n);

@@ -83,6 +83,8 @@ def _sig(name, res, args):
 _quant = _sig("csa_quant_kv", _i32, [_p, _i32, _i64, _i32, _i64, _i32, _p, _i64, _p])
 _index_ws = _sig("csa_index_workspace_size", ctypes.c_size_t, [ctypes.POINTER(IndexArgs)])
 _index = _sig("csa_index_topk", _i32, [ctypes.POINTER(IndexArgs), _p, ctypes.c_size_t, _p])
+_index_noalloc = _sig("csa_index_topk_noalloc", _i32, [ctypes.POINTER(IndexArgs), _p])
+_index_noalloc_cap = _sig("csa_index_noalloc_capacity", ctypes.c_size_t, [])
 _topk_ws = _sig("csa_topk_workspace_size", ctypes.c_size_t, [_i32, _i64])
 _topk = _sig("csa_topk_scores", _i32, [_p, _i32, _i64, _i64, _i32, _p, _p, ctypes.c_size_t, _p])
 _attn_ws = _sig("csa_attn_workspace_size", ctypes.c_size_t, [ctypes.POINTER(AttnArgs)])
@@ -98,7 +100,8 @@ _profile_collect = _sig("csa_profile_collect", _i32, [ctypes.POINTER(KernelTime)
 EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
-            "csa_profile_enable", "csa_profile_collect"]
+            "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc",
+            "csa_index_noalloc_capacity"]
 
 
 def profile_enable(on: bool) -> bool:
@@ -187,6 +190,16 @@ def csa_index_topk(args: IndexArgs, workspace=None, stream=None, device=None) ->
         workspace = _workspace(need, device or "cuda")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_index(ctypes.byref(args), _ptr(workspace), nbytes, _stream(stream)), "csa_index_topk")
+
+
+def csa_index_noalloc_capacity() -> int:
+    return int(_index_noalloc_cap())
+
+
+def csa_index_topk_noalloc(args: IndexArgs, stream=None) -> None:
+    """csa_index_topk with the library's fixed device scratch instead of a
+    caller workspace (see csa.h): for callers that cannot allocate."""
+    _check(_index_noalloc(ctypes.byref(args), _stream(stream)), "csa_index_topk_noalloc")
 
 
 def csa_topk_workspace_size(B: int, n: int) -> int:
