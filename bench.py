@@ -289,12 +289,13 @@ def run_gpu(args, cfg, rank, world, local_rank):
     value = tokens / (ms_max * 1e-3)
     alg = _algorithmic_bytes(cfg)
     # dominant kernel: the Full layer's indexer scoring over all T positions
-    name = "index_score_decode[full]"
+    name = "index_score_tc[full]" if "index_score_tc[full]" in kernels else "index_score_decode[full]"
     nl, tot = kernels.get(name, (0, 0.0))
     per_launch_ms = tot / nl if nl else float("nan")
     k_bytes = cfg.B * cfg.T * 64
     achieved = k_bytes / (per_launch_ms * 1e-3) / 1e9 if nl else None
-    src = os.path.join(ROOT, "indexer_selected_sparse_csa2_b200", "csrc", "index_decode.cu")
+    src = os.path.join(ROOT, "indexer_selected_sparse_csa2_b200", "csrc",
+                       "index_tc.cu" if name.startswith("index_score_tc") else "index_decode.cu")
     traffic = _traffic_record(src)
     line = {
         "metric": METRIC,

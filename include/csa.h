@@ -248,6 +248,10 @@ int32_t csa_profile_collect(csa_kernel_time* out, int32_t max_entries);
 
 /* ------------------------------------------------------------------------ */
 const char* csa_status_string(int32_t status);
+/* Device-side error code recorded by a kernel whose bounded wait on an
+ * mbarrier timed out (0 = none), then cleared.  Synchronises with the device
+ * (it copies the flag back); call it after the work it should cover. */
+int32_t csa_device_status(void);
 /* Number of kernels the library has enqueued since load (all entry points). */
 uint64_t csa_launch_count(void);
 int32_t csa_version(void);

@@ -93,6 +93,7 @@ _layer_ws = _sig("csa_layer_workspace_size", ctypes.c_size_t, [ctypes.POINTER(La
 _layer = _sig("csa_layer_step", _i32, [ctypes.POINTER(LayerDesc), _i32, _p, ctypes.c_size_t, _p])
 _status_string = _sig("csa_status_string", ctypes.c_char_p, [_i32])
 _launch_count = _sig("csa_launch_count", ctypes.c_uint64, [])
+_device_status = _sig("csa_device_status", _i32, [])
 _version = _sig("csa_version", _i32, [])
 _profile_enable = _sig("csa_profile_enable", _i32, [_i32])
 _profile_collect = _sig("csa_profile_collect", _i32, [ctypes.POINTER(KernelTime), _i32])
@@ -100,7 +101,7 @@ _profile_collect = _sig("csa_profile_collect", _i32, [ctypes.POINTER(KernelTime)
 EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
-            "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc",
+            "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
             "csa_index_noalloc_capacity"]
 
 
@@ -128,6 +129,11 @@ def status_string(status: int) -> str:
 
 def launch_count() -> int:
     return int(_launch_count())
+
+
+def device_status() -> int:
+    """Error code of a timed-out device wait since the last call (0 = none)."""
+    return int(_device_status())
 
 
 def version() -> int:

@@ -23,6 +23,7 @@ cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim
 size_t index_decode_ws_bytes(const csa_index_args* a);
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream);
 size_t attn_ws_bytes(const csa_attn_args* a);
+int read_tc_error(bool clear);
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream);
 
 static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -282,6 +283,8 @@ const char* csa_status_string(int32_t s) {
     default: return "unknown status";
   }
 }
+
+int32_t csa_device_status(void) { return (int32_t)read_tc_error(true); }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 int32_t csa_version(void) { return 1; }

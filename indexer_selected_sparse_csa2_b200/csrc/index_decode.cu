@@ -54,7 +54,7 @@ constexpr int kTilesPerIter = 4;                       // 4 x 16 rows per warp s
 constexpr int kRowsPerIter = 16 * kTilesPerIter;       // 64
 constexpr int kRowsPerCtaIter = kRowsPerIter * (kScoreThreads / 32);   // 512
 
-__global__ void __launch_bounds__(kScoreThreads) index_score_decode_kernel(ScoreParams p) {
+__global__ void __launch_bounds__(kScoreThreads, 2) index_score_decode_kernel(ScoreParams p) {
   __shared__ uint32_t h[kHistBins];
   __shared__ uint32_t hb[kHistBins];
   const int b = blockIdx.y;
@@ -80,27 +80,33 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_decode_kernel(Score
   float* sc = p.scores + (int64_t)b * p.n;
   __syncthreads();
 
-  for (int64_t base = lo + (int64_t)warp * kRowsPerIter; base < hi; base += kRowsPerCtaIter) {
-    uint4 ka[kTilesPerIter], kc[kTilesPerIter];
+  // Register double buffer: the loads of the warp's next 64 rows are issued
+  // before the current 64 rows are multiplied, so every warp keeps 4 KB of
+  // key reads in flight while it computes.
+  uint4 ka[2][kTilesPerIter], kc[2][kTilesPerIter];
+  auto load = [&](int buf, int64_t base) {
 #pragma unroll
     for (int u = 0; u < kTilesPerIter; ++u) {
       const int64_t r0 = base + 16 * u + g, r1 = r0 + 8;
-      ka[u] = make_uint4(0, 0, 0, 0);
-      kc[u] = make_uint4(0, 0, 0, 0);
+      ka[buf][u] = make_uint4(0, 0, 0, 0);
+      kc[buf][u] = make_uint4(0, 0, 0, 0);
       if (r0 < hi) {
         const int64_t s0 = pl ? (int64_t)pl[r0] : r0;
-        ka[u] = ld_nc_v4(kb + s0 * p.key_row_stride + 16 * t);
+        ka[buf][u] = ld_nc_v4(kb + s0 * p.key_row_stride + 16 * t);
       }
       if (r1 < hi) {
         const int64_t s1 = pl ? (int64_t)pl[r1] : r1;
-        kc[u] = ld_nc_v4(kb + s1 * p.key_row_stride + 16 * t);
+        kc[buf][u] = ld_nc_v4(kb + s1 * p.key_row_stride + 16 * t);
       }
     }
+  };
+  auto compute = [&](int buf, int64_t base) {
 #pragma unroll
     for (int u = 0; u < kTilesPerIter; ++u) {
       float c[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_e4m3_16832(c, ka[u].x, kc[u].x, ka[u].y, kc[u].y, qf[0], qf[1]);
-      mma_e4m3_16832(c, ka[u].z, kc[u].z, ka[u].w, kc[u].w, qf[2], qf[3]);
+      const uint4 A = ka[buf][u], C = kc[buf][u];
+      mma_e4m3_16832(c, A.x, C.x, A.y, C.y, qf[0], qf[1]);
+      mma_e4m3_16832(c, A.z, C.z, A.w, C.w, qf[2], qf[3]);
       float s_lo = w0 * fmaxf(c[0], 0.f) + w1 * fmaxf(c[1], 0.f);   // row g
       float s_hi = w0 * fmaxf(c[2], 0.f) + w1 * fmaxf(c[3], 0.f);   // row g + 8
       s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
@@ -144,6 +150,20 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_decode_kernel(Score
         }
       }
     }
+  };
+  // two iterations per loop trip so that the buffer index is a constant
+  int64_t base = lo + (int64_t)warp * kRowsPerIter;
+  if (base < hi) load(0, base);
+  while (base < hi) {
+    int64_t next = base + kRowsPerCtaIter;
+    if (next < hi) load(1, next);
+    compute(0, base);
+    base = next;
+    if (base >= hi) break;
+    next = base + kRowsPerCtaIter;
+    if (next < hi) load(0, next);
+    compute(1, base);
+    base = next;
   }
   __syncthreads();
   uint32_t* gh = p.hist + (int64_t)b * kHistBins;
@@ -155,7 +175,8 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_decode_kernel(Score
 }
 
 int64_t score_chunk(int B, int64_t n) {
-  int64_t target = (int64_t)kNumSMs * 4 / (B > 0 ? B : 1);
+  // one wave: two resident CTAs per SM over all rows
+  int64_t target = ((int64_t)kNumSMs * 2 + B - 1) / (B > 0 ? B : 1);
   if (target < 1) target = 1;
   int64_t c = (n + target - 1) / target;
   c = (c + kRowsPerCtaIter - 1) / kRowsPerCtaIter * kRowsPerCtaIter;
@@ -182,6 +203,9 @@ struct IndexWs {
 };
 
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
+                            int64_t nb, cudaStream_t stream);
 
 // Workspace layout of one decode index call.
 static IndexWs carve_index_ws(const csa_index_args* a, void* ws) {
@@ -234,7 +258,10 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     p.nb = (a->T + a->pool_block_len - 1) / a->pool_block_len;
     p.block_len = a->pool_block_len;
   }
-  e = launch_score_decode(p, B, stream);
+  // full scans run on the tcgen05 scorer; pool searches gather rows and use
+  // the mma.sync scorer
+  if (a->pool) e = launch_score_decode(p, B, stream);
+  else e = launch_score_tc(a, p.scores, p.hist, p.bmax, p.bhist, p.nb, stream);
   if (e != cudaSuccess) return e;
 
   SelectJob jobs[2];

@@ -21,10 +21,12 @@
 
 namespace csa {
 
-constexpr int kExtractThreads = 256;
+constexpr int kExtractThreads = 256;     // 8 warps = 8 consecutive runs per CTA
+constexpr int kRunsPerCta = kExtractThreads / 32;
 constexpr int kFinalThreads = 1024;
-constexpr int kFinalSmemCap = 12288;    // candidates staged in shared memory
-constexpr int kMaxChunks = 1024;
+constexpr int kListCap = 20480;          // candidates staged in shared memory
+constexpr int kMaxRuns = 8192;
+constexpr int kRunsPerThread = kMaxRuns / kFinalThreads;
 
 struct SelectJobs {
   SelectJob j[2];
@@ -32,17 +34,17 @@ struct SelectJobs {
 
 SelectPlan plan_select(int B, int64_t n) {
   SelectPlan p;
-  // ~2 waves of extract CTAs over all rows; at least 4096 slots per CTA; at
-  // most kMaxChunks runs per row so the final CTA can scan the run counts.
-  int64_t target = (int64_t)kNumSMs * 4 / (B > 0 ? B : 1);
-  if (target < 1) target = 1;
-  int64_t chunk = (n + target - 1) / target;
-  if (chunk < 4096) chunk = 4096;
-  int64_t minc = (n + kMaxChunks - 1) / kMaxChunks;
-  if (chunk < minc) chunk = minc;
-  chunk = (chunk + 255) / 256 * 256;
-  p.chunk = chunk;
-  p.nchunks = (int)((n + chunk - 1) / chunk);
+  // about four resident extract CTAs per SM over all rows; each warp scans
+  // one run of at least 512 slots; at most kMaxRuns runs per row.
+  int64_t ctas = ((int64_t)kNumSMs * 4 + B - 1) / (B > 0 ? B : 1);
+  if (ctas < 1) ctas = 1;
+  int64_t run = (n + ctas * kRunsPerCta - 1) / (ctas * kRunsPerCta);
+  if (run < 512) run = 512;
+  const int64_t minr = (n + kMaxRuns - 1) / kMaxRuns;
+  if (run < minr) run = minr;
+  run = (run + 127) / 128 * 128;
+  p.chunk = run;
+  p.nchunks = (int)((n + run - 1) / run);
   if (p.nchunks < 1) p.nchunks = 1;
   return p;
 }
@@ -97,13 +99,13 @@ __global__ void __launch_bounds__(256) select_hist_kernel(SelectJobs jobs) {
   const SelectJob& J = jobs.j[blockIdx.z];
   const int b = blockIdx.y;
   const int c = blockIdx.x;
-  if (c >= J.nchunks) return;
+  if (c * kRunsPerCta >= J.nchunks) return;
   __shared__ uint32_t h[kHistBins];
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) h[i] = 0;
   __syncthreads();
   const int64_t nrow = J.n_row ? (int64_t)min((int64_t)J.n_row[b], J.n) : J.n;
-  const int64_t lo = (int64_t)c * J.chunk;
-  const int64_t hi = min(lo + J.chunk, nrow);
+  const int64_t lo = (int64_t)c * kRunsPerCta * J.chunk;
+  const int64_t hi = min(lo + kRunsPerCta * J.chunk, nrow);
   const float* v = J.vals + (int64_t)b * J.row_stride;
   for (int64_t s = lo + threadIdx.x; s < hi; s += blockDim.x) atomicAdd(&h[order_key(v[s]) >> (32 - kHistBits)], 1u);
   __syncthreads();
@@ -166,39 +168,65 @@ CSA_DEV int threshold_bin(const uint32_t* gh, int K, uint32_t* warp_tot, uint32_
   return *out_bin;
 }
 
+// Each warp scans one run of slots in order, 4 slots per lane per step, and
+// appends the run's candidates (bin >= beta) to the run's own region of the
+// candidate buffer, keeping slot order (lane-order prefix via shuffles).
+template <bool VEC>
 __global__ void __launch_bounds__(kExtractThreads) select_extract_kernel(SelectJobs jobs) {
   const SelectJob& J = jobs.j[blockIdx.z];
   const int b = blockIdx.y;
-  const int c = blockIdx.x;
-  if (c >= J.nchunks) return;
+  if ((int)blockIdx.x * kRunsPerCta >= J.nchunks) return;
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t total;
   __shared__ int bin;
   const int beta = threshold_bin(J.hist + (int64_t)b * kHistBins, J.K, warp_tot, &total, &bin);
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kRunsPerCta + (threadIdx.x >> 5);
+  if (r >= J.nchunks) return;
   const int64_t nrow = J.n_row ? (int64_t)min((int64_t)J.n_row[b], J.n) : J.n;
-  const int64_t lo = (int64_t)c * J.chunk;
+  const int64_t lo = (int64_t)r * J.chunk;
   const int64_t hi = min(lo + J.chunk, nrow);
   const float* v = J.vals + (int64_t)b * J.row_stride;
   uint32_t* ck = J.cand_key + (int64_t)b * J.n + lo;
   int32_t* cp = J.cand_pos + (int64_t)b * J.n + lo;
   uint32_t run = 0;
-  for (int64_t s0 = lo; s0 < hi; s0 += kExtractThreads) {
-    const int64_t s = s0 + threadIdx.x;
-    uint32_t key = 0;
-    uint32_t f = 0;
-    if (s < hi) {
-      key = order_key(v[s]);
-      f = (int)(key >> (32 - kHistBits)) >= beta;
+  for (int64_t s0 = lo; s0 < hi; s0 += 128) {
+    const int64_t s = s0 + 4 * lane;
+    float x[4];
+    if (VEC && s + 3 < hi) {
+      const float4 f = *reinterpret_cast<const float4*>(v + s);
+      x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = s + k < hi ? v[s + k] : 0.f;
     }
-    const uint32_t incl = block_incl_scan<kExtractThreads>(f, warp_tot, &total);
-    if (f) {
-      ck[run + incl - 1] = key;
-      cp[run + incl - 1] = (int32_t)s;
+    uint32_t key[4];
+    uint32_t flags = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      key[k] = order_key(x[k]);
+      if (s + k < hi && (int)(key[k] >> (32 - kHistBits)) >= beta) flags |= 1u << k;
     }
-    run += total;
-    __syncthreads();
+    const uint32_t c = __popc(flags);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t at = run + incl - c;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (flags & (1u << k)) {
+        ck[at] = key[k];
+        cp[at] = (int32_t)(s + k);
+        ++at;
+      }
+    }
+    run += tot;
   }
-  if (threadIdx.x == 0) J.cnt[(int64_t)b * J.nchunks + c] = (int32_t)run;
+  if (lane == 0) J.cnt[(int64_t)b * J.nchunks + r] = (int32_t)run;
 }
 
 // ----------------------------------------------------------------- final --
@@ -219,40 +247,59 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs 
   const SelectJob& J = jobs.j[blockIdx.y];
   const int b = blockIdx.x;
   extern __shared__ __align__(16) uint8_t smem[];
-  uint32_t* skey = reinterpret_cast<uint32_t*>(smem);
-  int32_t* spos = reinterpret_cast<int32_t*>(smem + kFinalSmemCap * 4);
-  __shared__ uint32_t offs[kMaxChunks];
+  uint32_t* offs = reinterpret_cast<uint32_t*>(smem);                       // [kMaxRuns]
+  uint32_t* skey = offs + kMaxRuns;                                          // [kListCap]
+  int32_t* spos = reinterpret_cast<int32_t*>(skey + kListCap);               // [kListCap]
   __shared__ uint32_t warp_tot[32];
   __shared__ uint32_t total;
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_krem;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nruns = J.nchunks;
+  const int32_t* cnt_row = J.cnt + (int64_t)b * nruns;
 
-  // 1. run offsets
-  const int tid = threadIdx.x;
-  uint32_t cnt = tid < J.nchunks ? (uint32_t)J.cnt[(int64_t)b * J.nchunks + tid] : 0u;
-  const uint32_t incl = block_incl_scan<kFinalThreads>(cnt, warp_tot, &total);
-  offs[tid] = incl - cnt;
+  // 1. run offsets (thread t owns runs [8t, 8t + 8))
+  uint32_t c8[kRunsPerThread];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int k = 0; k < kRunsPerThread; ++k) {
+    const int r = kRunsPerThread * tid + k;
+    c8[k] = r < nruns ? (uint32_t)cnt_row[r] : 0u;
+    mine += c8[k];
+  }
+  const uint32_t incl = block_incl_scan<kFinalThreads>(mine, warp_tot, &total);
   const uint32_t m = total;
-  __syncthreads();
-
-  // 2. contiguous ordered list (shared memory when it fits)
-  const bool in_smem = m <= (uint32_t)kFinalSmemCap;
-  uint32_t* lk = in_smem ? skey : J.list_key + (int64_t)b * J.n;
-  int32_t* lp = in_smem ? spos : J.list_pos + (int64_t)b * J.n;
-  for (int c = 0; c < J.nchunks; ++c) {
-    const uint32_t n_c = (uint32_t)J.cnt[(int64_t)b * J.nchunks + c];
-    const uint32_t* src_k = J.cand_key + (int64_t)b * J.n + (int64_t)c * J.chunk;
-    const int32_t* src_p = J.cand_pos + (int64_t)b * J.n + (int64_t)c * J.chunk;
-    for (uint32_t i = tid; i < n_c; i += kFinalThreads) {
-      lk[offs[c] + i] = src_k[i];
-      lp[offs[c] + i] = src_p[i];
+  {
+    uint32_t o = incl - mine;
+#pragma unroll
+    for (int k = 0; k < kRunsPerThread; ++k) {
+      offs[kRunsPerThread * tid + k] = o;
+      o += c8[k];
     }
   }
   __syncthreads();
 
-  // 3. exact threshold by 4 passes of an 8-bit radix select
+  // 2. contiguous ordered list (shared memory when it fits); warp w copies
+  //    runs w, w + 32, ...
+  const bool in_smem = m <= (uint32_t)kListCap;
+  uint32_t* lk = in_smem ? skey : J.list_key + (int64_t)b * J.n;
+  int32_t* lp = in_smem ? spos : J.list_pos + (int64_t)b * J.n;
+  for (int r = warp; r < nruns; r += kFinalThreads / 32) {
+    const uint32_t n_r = (uint32_t)cnt_row[r];
+    const uint32_t* src_k = J.cand_key + (int64_t)b * J.n + (int64_t)r * J.chunk;
+    const int32_t* src_p = J.cand_pos + (int64_t)b * J.n + (int64_t)r * J.chunk;
+    const uint32_t o = offs[r];
+    for (uint32_t i = lane; i < n_r; i += 32) {
+      lk[o + i] = src_k[i];
+      lp[o + i] = src_p[i];
+    }
+  }
+  __syncthreads();
+
+  // 3. exact threshold tau by 4 passes of an 8-bit radix select, and the
+  //    number of slots equal to tau that the Top-K still needs
   const uint32_t K = (uint32_t)J.K;
-  bool take_all = m <= K;
+  const bool take_all = m <= K;
   if (tid == 0) { s_prefix = 0; s_krem = K; }
   __syncthreads();
   if (!take_all) {
@@ -298,30 +345,43 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs 
     }
   }
   const uint32_t tau = s_prefix;
-  const uint32_t need_eq = s_krem;   // slots equal to tau to take (lowest first)
+  const uint32_t need_eq = s_krem;   // slots equal to tau to take, lowest first
 
-  // 4. ordered emission
-  uint32_t eq_base = 0, out_base = 0;
-  for (uint32_t i0 = 0; i0 < m; i0 += kFinalThreads) {
-    const uint32_t i = i0 + tid;
-    uint32_t k = 0;
-    bool valid = i < m;
-    if (valid) k = lk[i];
-    const uint32_t is_eq = (valid && !take_all && k == tau) ? 1u : 0u;
-    const uint32_t eq_incl = block_incl_scan<kFinalThreads>(is_eq, warp_tot, &total);
-    const uint32_t eq_tot = total;
-    const bool sel = valid && (take_all || k > tau || (is_eq && eq_base + eq_incl - 1 < need_eq));
-    const uint32_t s_incl = block_incl_scan<kFinalThreads>(sel ? 1u : 0u, warp_tot, &total);
-    const uint32_t s_tot = total;
-    if (sel) write_selected(J, b, out_base + s_incl - 1, lp[i]);
-    eq_base += eq_tot;
-    out_base += s_tot;
-    __syncthreads();
+  // 4. ordered emission: thread t owns the contiguous segment
+  //    [t*seg, (t+1)*seg) of the list
+  const uint32_t seg = (m + kFinalThreads - 1) / kFinalThreads;
+  const uint32_t i0 = min(m, tid * seg), i1 = min(m, i0 + seg);
+  uint32_t n_eq = 0;
+  if (!take_all)
+    for (uint32_t i = i0; i < i1; ++i) n_eq += lk[i] == tau ? 1u : 0u;
+  const uint32_t eq_excl = block_incl_scan<kFinalThreads>(n_eq, warp_tot, &total) - n_eq;
+  uint32_t n_sel = 0;
+  {
+    uint32_t eq_rank = eq_excl;
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint32_t k = lk[i];
+      bool sel = take_all || k > tau;
+      if (!take_all && k == tau) { sel = eq_rank < need_eq; ++eq_rank; }
+      n_sel += sel ? 1u : 0u;
+    }
   }
+  const uint32_t sel_incl = block_incl_scan<kFinalThreads>(n_sel, warp_tot, &total);
+  const uint32_t out_count = total;
+  {
+    uint32_t j = sel_incl - n_sel;
+    uint32_t eq_rank = eq_excl;
+    for (uint32_t i = i0; i < i1; ++i) {
+      const uint32_t k = lk[i];
+      bool sel = take_all || k > tau;
+      if (!take_all && k == tau) { sel = eq_rank < need_eq; ++eq_rank; }
+      if (sel) write_selected(J, b, j++, lp[i]);
+    }
+  }
+
   // 5. padding and valid length
   const int32_t width = J.out_width;
   int32_t* out = J.out + (int64_t)b * J.out_stride;
-  const int64_t written = (int64_t)out_base * (J.expand ? J.expand : 1);
+  const int64_t written = (int64_t)out_count * (J.expand ? J.expand : 1);
   for (int64_t j = written + tid; j < width; j += kFinalThreads) out[j] = -1;
   __syncthreads();
   if (J.expand && J.out_len && tid == 0) {
@@ -338,7 +398,12 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
   js.j[0] = jobs[0];
   js.j[1] = njobs > 1 ? jobs[1] : jobs[0];
   int maxc = 0;
-  for (int i = 0; i < njobs; ++i) maxc = jobs[i].nchunks > maxc ? jobs[i].nchunks : maxc;
+  bool vec = true;
+  for (int i = 0; i < njobs; ++i) {
+    const int ctas = (jobs[i].nchunks + kRunsPerCta - 1) / kRunsPerCta;
+    maxc = ctas > maxc ? ctas : maxc;
+    vec = vec && (((uintptr_t)jobs[i].vals & 15) == 0) && (jobs[i].row_stride % 4 == 0);
+  }
   dim3 g(maxc, B, njobs);
   if (build_hist) {
     ProfScope ps(stream, "select_hist");
@@ -347,9 +412,10 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
   }
   {
     ProfScope ps(stream, "select_extract");
-    select_extract_kernel<<<g, kExtractThreads, 0, stream>>>(js);
+    if (vec) select_extract_kernel<true><<<g, kExtractThreads, 0, stream>>>(js);
+    else select_extract_kernel<false><<<g, kExtractThreads, 0, stream>>>(js);
   }
-  const size_t smem = (size_t)kFinalSmemCap * 8;
+  const size_t smem = (size_t)kMaxRuns * 4 + (size_t)kListCap * 8;
   static bool attr_set = false;
   if (!attr_set) {
     cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -18,9 +18,9 @@ struct SelectJob {
   int32_t* cand_pos;        // [B][n]
   uint32_t* list_key;       // [B][n] ordered contiguous copy (used when the list exceeds smem)
   int32_t* list_pos;        // [B][n]
-  int32_t* cnt;             // [B][nchunks]
-  int64_t chunk;            // slots per extract CTA
-  int nchunks;
+  int32_t* cnt;             // [B][nchunks] candidates found in each run
+  int64_t chunk;            // slots per run (one warp of an extract CTA scans one run)
+  int nchunks;              // runs per row (<= 8192)
   // output
   int32_t* out;             // [B][out_stride]
   int64_t out_stride;

@@ -170,3 +170,9 @@ def test_topk_scores_candidate_overflow_path(csa):
     s[0, 1000:1100] = 1.0
     got = _run_topk(csa, s, K)
     assert np.array_equal(got[0], oi.topk(s[0].astype(np.float64), K))
+
+
+def test_zz_no_device_wait_timeouts(csa):
+    """No bounded device wait of the kernels above ran out (status 0)."""
+    torch.cuda.synchronize()
+    assert csa.device_status() == 0
