@@ -110,8 +110,7 @@ csa_status csa_quant_kv(const void* src, int32_t src_dtype, int64_t n_rows, int3
 typedef struct {
   int32_t B;                 /* sequences, >= 1 */
   int32_t n_q;               /* query tokens per sequence, >= 1 */
-  int64_t T;                 /* cache length, n_q <= T < 2^31 (n_q > 1:
-                                CSA_ERR_UNSUPPORTED in this version) */
+  int64_t T;                 /* cache length, n_q <= T < 2^31 */
   int32_t H_I;               /* indexer heads, 1..8 */
   int32_t d_I;               /* indexer head dim; must be 64 */
   const uint8_t* keys;       /* E4M3 key of position s of sequence b at
@@ -120,7 +119,7 @@ typedef struct {
   int64_t key_batch_stride;  /* bytes, multiple of 16 */
   const uint8_t* q;          /* E4M3 [B][n_q][H_I][64], contiguous */
   const float* w;            /* fp32 [B][n_q][H_I], contiguous */
-  int32_t K;                 /* 1..65536 */
+  int32_t K;                 /* 1..65536 (1..4096 when n_q > 1) */
   const int32_t* pool;       /* optional [B][pool_cap] ascending positions */
   const int32_t* pool_len;   /* [B] valid entries of pool (required with pool) */
   int32_t pool_cap;          /* row length of pool */

@@ -24,6 +24,7 @@ size_t index_decode_ws_bytes(const csa_index_args* a);
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream);
 size_t attn_ws_bytes(const csa_attn_args* a);
 int read_tc_error(bool clear);
+int read_pf_error(bool clear);
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream);
 
 static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -60,8 +61,10 @@ static csa_status check_index(const csa_index_args* a) {
   if (!al16(a->keys) || !al16i(a->key_row_stride) || !al16i(a->key_batch_stride) || !al16(a->q))
     return CSA_ERR_ALIGNMENT;
   if (a->n_q > 1) {
+    // prefill chunk: no pool, no score output, K within the final select's capacity
     if (a->pool || a->pool_out || a->scores) return CSA_ERR_UNSUPPORTED;
-    return CSA_ERR_UNSUPPORTED;   // prefill scoring is provided by the GEMM path
+    if (a->K > 4096) return CSA_ERR_SHAPE;
+    return CSA_OK;
   }
   if (a->pool && a->pool_out) return CSA_ERR_UNSUPPORTED;
   if (a->pool) {
@@ -284,7 +287,10 @@ const char* csa_status_string(int32_t s) {
   }
 }
 
-int32_t csa_device_status(void) { return (int32_t)read_tc_error(true); }
+int32_t csa_device_status(void) {
+  const int a = read_tc_error(true), b = read_pf_error(true);
+  return (int32_t)(a ? a : b);
+}
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 int32_t csa_version(void) { return 1; }

@@ -225,9 +225,16 @@ static IndexWs carve_index_ws(const csa_index_args* a, void* ws) {
   return w;
 }
 
-size_t index_decode_ws_bytes(const csa_index_args* a) { return carve_index_ws(a, nullptr).bytes; }
+size_t index_prefill_ws_bytes(const csa_index_args* a);
+cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t stream);
+
+size_t index_decode_ws_bytes(const csa_index_args* a) {
+  if (a->n_q > 1) return index_prefill_ws_bytes(a);
+  return carve_index_ws(a, nullptr).bytes;
+}
 
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream) {
+  if (a->n_q > 1) return run_index_prefill(a, ws, stream);
   IndexWs w = carve_index_ws(a, ws);
   const int B = a->B;
   const int64_t n = a->pool ? (int64_t)a->pool_cap : a->T;
