@@ -334,9 +334,65 @@ def run_gpu(args, cfg, rank, world, local_rank):
                 "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4)},
         "clocks": clk,
     }
+    if world == 1 and not args.no_prefill:
+        del dc, descs, ws
+        torch.cuda.empty_cache()
+        line["prefill"] = run_prefill(args, dev)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds_budget=args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def run_prefill(args, dev):
+    """One prefill chunk (4096 causal queries at a 2^20-token cache): the
+    step's FP4 / FP8 encodes of the new tokens, the FP8 tcgen05 indexer GEMM
+    with exact per-query Top-K, and attention for every query."""
+    import torch
+    import indexer_selected_sparse_csa2_b200 as csa
+    from csa_synth import get_config
+    from csa_synth.device import DeviceCase
+    cfg = get_config("prefill_1m")
+    dc = DeviceCase(cfg, device=dev)
+    descs = dc.layer_descs(append_rows=True)
+    ws = torch.empty(max(csa.csa_layer_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.prefill_warmup):
+        csa.csa_layer_step(descs, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    csa.profile_enable(True)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.prefill_steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.prefill_steps)]
+    for i in range(args.prefill_steps):
+        starts[i].record(stream)
+        csa.csa_layer_step(descs, workspace=ws, stream=stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    csa.profile_enable(False)
+    kern = csa.profile_collect()
+    assert csa.device_status() == 0
+    ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.prefill_steps
+    _, bf16_peak, peak_kind = _peaks()
+    fp8_peak = 2.0 * bf16_peak
+    P = cfg.T - cfg.n_q
+    # dense indexer work: n_q x 8 heads x 64 x (keys visible to each query) x 2
+    flops = sum(2.0 * cfg.H_I * cfg.d_I * (P + t + 1) for t in range(cfg.n_q))
+    nl, tot = kern.get("prefill_score_tc[main]", (0, 0.0))
+    main_ms = tot / nl if nl else float("nan")
+    tflops = flops / (main_ms * 1e-3) / 1e12 if nl else None
+    attn_flops = 2.0 * 2.0 * cfg.n_q * cfg.H * cfg.D * (cfg.K + cfg.n_win)
+    return {
+        "workload": "prefill_1m", "n_q": cfg.n_q, "T": cfg.T, "K": cfg.K, "W": cfg.W,
+        "ms_per_chunk": round(ms, 3), "tokens_per_s": round(cfg.n_q / (ms * 1e-3), 1),
+        "index_gemm": {"bound": "tensor", "achieved": round(tflops, 1) if tflops else None,
+                       "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                       "frac": round(tflops / fp8_peak, 4) if tflops else None,
+                       "flops_per_launch": flops, "launch_ms": round(main_ms, 4),
+                       "peak_kind": f"{peak_kind} bf16 x 2 (FP8 / BF16 dense ratio)"},
+        "attention_tflops": round(attn_flops / (kern.get("sparse_attn_mma", (1, float("nan")))[1] /
+                                                max(1, args.prefill_steps) * 1e-3) / 1e12, 1),
+        "kernels": {k: {"launches": v[0], "ms_per_chunk": round(v[1] / args.prefill_steps, 4)}
+                    for k, v in kern.items()},
+    }
 
 
 def main():
@@ -348,6 +404,9 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=30.0)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=3)
+    ap.add_argument("--prefill-warmup", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -118,22 +118,39 @@ class DeviceCase:
             dl = self.layers[li]
             o = L.owner
             if append_rows:
+                # the step's new tokens: position T-1 of every sequence at decode
+                # (rows strided by the batch stride), positions [T-n_q, T) of the
+                # single sequence of a prefill chunk
+                n_new = cfg.n_q
+                if n_new > 1 and cfg.B != 1:
+                    raise ValueError("prefill appends are built for one sequence")
                 jobs = []
+                t_new = cfg.T - n_new
                 if o == li:
-                    mx = torch.stack([self._latent_tensor(wl.main_latent(cfg, o, b, cfg.T - 1, 1))[0]
-                                      for b in range(cfg.B)])
-                    kx = torch.from_numpy(np.stack([wl.index_key(cfg, o, b, cfg.T - 1, 1)[0]
-                                                    for b in range(cfg.B)])).to(self.device)
-                    kvrow = self.kv[o][:, cfg.T - 1]
-                    krow = self.keys[o][:, cfg.T - 1]
-                    jobs.append(csa.quant_job(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kvrow,
-                                              self.kv[o].stride(0)))
-                    jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, self.keys[o].stride(0)))
+                    if n_new == 1:
+                        mx = torch.stack([self._latent_tensor(wl.main_latent(cfg, o, b, cfg.T - 1, 1))[0]
+                                          for b in range(cfg.B)])
+                        kx = torch.from_numpy(np.stack([wl.index_key(cfg, o, b, cfg.T - 1, 1)[0]
+                                                        for b in range(cfg.B)])).to(self.device)
+                        kvrow, krow = self.kv[o][:, cfg.T - 1], self.keys[o][:, cfg.T - 1]
+                        kv_stride, k_stride = self.kv[o].stride(0), self.keys[o].stride(0)
+                    else:
+                        mx = self._latent_tensor(wl.main_latent(cfg, o, 0, t_new, n_new))
+                        kx = torch.from_numpy(wl.index_key(cfg, o, 0, t_new, n_new)).to(self.device)
+                        kvrow, krow = self.kv[o][0, t_new:], self.keys[o][0, t_new:]
+                        kv_stride, k_stride = self.kv[o].stride(1), self.keys[o].stride(1)
+                    jobs.append(csa.quant_job(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kvrow, kv_stride))
+                    jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, k_stride))
                     self._append_src += [mx, kx]
-                wx = torch.stack([self._latent_tensor(wl.window_latent(cfg, li, b))[cfg.win_rows - 1]
-                                  for b in range(cfg.B)])
-                wrow = dl.win[:, cfg.win_rows - 1]
-                jobs.append(csa.quant_job(wx, csa.CSA_FMT_FP8_E4M3_UE8M0X32, wrow, dl.win.stride(0)))
+                r0 = cfg.win_rows - n_new
+                if n_new == 1:
+                    wx = torch.stack([self._latent_tensor(wl.window_latent(cfg, li, b))[r0]
+                                      for b in range(cfg.B)])
+                    wrow, w_stride = dl.win[:, r0], dl.win.stride(0)
+                else:
+                    wx = self._latent_tensor(wl.window_latent(cfg, li, 0)[r0:])
+                    wrow, w_stride = dl.win[0, r0:], dl.win.stride(1)
+                jobs.append(csa.quant_job(wx, csa.CSA_FMT_FP8_E4M3_UE8M0X32, wrow, w_stride))
                 self._append_src.append(wx)
                 for k, j in enumerate(jobs):
                     d.append[k] = j
@@ -145,5 +162,6 @@ class DeviceCase:
             d.attn = csa.attn_args(q=dl.q, kv=self.kv[o], idx=None, win=dl.win, n_win=cfg.n_win,
                                    softmax_scale=cfg.softmax_scale, out=dl.out, lse=dl.lse, sink=dl.sink,
                                    K=0)
+            d._keep = (getattr(d, "_keep", None), self.keys, self.kv, dl)
             descs.append(d)
         return csa.make_layer_array(descs)

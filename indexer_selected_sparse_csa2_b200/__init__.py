@@ -235,9 +235,13 @@ def csa_sparse_attn(args: AttnArgs, workspace=None, stream=None, device=None) ->
 
 
 def make_layer_array(layers: Sequence[LayerDesc]):
+    """ctypes array of LayerDesc.  Assigning an IndexArgs / AttnArgs /
+    QuantJob into a LayerDesc copies raw pointers only: the caller keeps the
+    tensors they point at alive (attach them to the LayerDesc as `_keep`)."""
     arr = (LayerDesc * len(layers))()
     for i, L in enumerate(layers):
         arr[i] = L
+    arr._keep = list(layers)
     return arr
 
 
@@ -274,6 +278,8 @@ def index_args(*, keys, q, w, K: int, idx, T: Optional[int] = None, n_q: int = 1
     a.pool_blocks, a.pool_block_len = pool_blocks, pool_block_len
     a.idx = _ptr(idx)
     a.scores = _ptr(scores)
+    # the struct holds raw device pointers: keep the tensors alive with it
+    a._keep = (keys, q, w, pool, pool_len, pool_out, pool_out_len, idx, scores)
     return a
 
 
@@ -292,6 +298,7 @@ def attn_args(*, q, kv, idx, win, n_win: int, softmax_scale: float, out, lse=Non
     a.n_win = n_win
     a.softmax_scale = softmax_scale
     a.sink, a.out, a.lse = _ptr(sink), _ptr(out), _ptr(lse)
+    a._keep = (q, kv, idx, win, out, lse, sink)
     return a
 
 
@@ -306,4 +313,5 @@ def quant_job(src, fmt: int, dst, dst_row_stride: int, n_rows: Optional[int] = N
     j.fmt = fmt
     j.dst = _ptr(dst)
     j.dst_row_stride = dst_row_stride
+    j._keep = (src, dst)
     return j

@@ -12,7 +12,9 @@
 //      those scores; a Top-r select per query gives a threshold tau_t (the
 //      r-th best sampled score), chosen so that ~2K positions should pass;
 //   2  main pass: every (t, s) with S >= tau_t is appended (order key,
-//      position) to query t's candidate buffer;
+//      position) to query t's candidate region for that key chunk; each
+//      (query block, key chunk) belongs to one CTA, so the append cursor is a
+//      shared-memory counter (no global atomic round trip per hit);
 //   3  final: per query, if its candidates provably contain the Top-K (at
 //      least K of them, or tau = -inf, and no overflow) an exact radix select
 //      with lowest-position tie-break runs on them; otherwise an exact
@@ -31,7 +33,8 @@ constexpr int kPfAcc = 2;
 constexpr int kPfEpiWarps = 16;                       // 4 TMEM quarters x 4 query groups of 8
 constexpr int kPfThreads = 64 + 32 * kPfEpiWarps;     // 576
 constexpr int kSampleStride = 64;                     // sample every 64th key tile
-constexpr int kCandCap = 16384;                       // candidates kept per query
+constexpr int kCandCap = 16384;                       // candidates the final select holds per query
+constexpr int kChunkCap = 8192;                       // candidates kept per (query, key chunk)
 constexpr int kPfChunkTiles = 1024;                   // key tiles per work item
 
 static __device__ int g_pf_error;
@@ -49,8 +52,8 @@ struct PfParams {
   float* sample;           // [B*n_q][n_samp]    (mode 0)
   int64_t n_samp;
   const float* tau;        // [B*n_q]           (mode 1)
-  uint2* cand;             // [B*n_q][kCandCap] (mode 1): (order key, position)
-  uint32_t* cnt;           // [B*n_q]
+  uint2* cand;             // [B*n_q][kchunks][kChunkCap] (mode 1): (order key, position)
+  uint32_t* cnt;           // [B*n_q][kchunks] hits per (query, key chunk), overflow included
 };
 
 struct PfSmem {
@@ -144,6 +147,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
   int64_t run = 0;
   bool failed = false;                 // this thread saw a wait time out
   __shared__ int any_failed;           // block-uniform copy, read after barriers
+  __shared__ uint32_t s_cnt[kPfQPerBlock];
   if (tid == 0) any_failed = 0;
   for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
     const PfItem x = pf_item(p, it);
@@ -162,6 +166,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
       const int t = x.qb * kPfQPerBlock + qq;
       S.wts[i] = (j < p.H_I && t < p.n_q) ? p.w[((int64_t)x.b * p.n_q + t) * p.H_I + j] : 0.f;
     }
+    if (tid < kPfQPerBlock) s_cnt[tid] = 0;
     fence_proxy_async_smem();
     __syncthreads();
 
@@ -208,6 +213,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
 #pragma unroll
       for (int k = 0; k < 8; ++k) tau[k] = (p.mode == 1 && k < nlive) ? p.tau[row0 + k] : 0.f;
       const float* wq = S.wts + qg * 64;
+      const int kc = (int)(x.kt0 / kPfChunkTiles);
       for (int64_t i = 0; i < n_t && !failed; ++i) {
         const int64_t g = run + i;
         const int a = (int)(g % kPfAcc);
@@ -240,9 +246,9 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
               const int64_t col = (tile / kSampleStride) * kPfRows + 32 * quarter + lane;
               p.sample[(row0 + k) * p.n_samp + col] = vis ? sc : -INFINITY;
             } else if (vis && sc >= tau[k]) {
-              const uint32_t slot = atomicAdd(&p.cnt[row0 + k], 1u);
-              if (slot < (uint32_t)kCandCap)
-                p.cand[(row0 + k) * kCandCap + slot] = make_uint2(order_key(sc), (uint32_t)pos);
+              const uint32_t slot = atomicAdd(&s_cnt[qg * 8 + k], 1u);
+              if (slot < (uint32_t)kChunkCap)
+                p.cand[((row0 + k) * p.kchunks + kc) * kChunkCap + slot] = make_uint2(order_key(sc), (uint32_t)pos);
             }
           }
         }
@@ -251,6 +257,10 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
     run += n_t;
     if (failed) atomicExch(&any_failed, 1);
     __syncthreads();
+    if (p.mode == 1 && tid < kPfQPerBlock) {
+      const int t = x.qb * kPfQPerBlock + tid;
+      if (t < p.n_q) p.cnt[((int64_t)x.b * p.n_q + t) * p.kchunks + x.kt0 / kPfChunkTiles] = s_cnt[tid];
+    }
     if (any_failed) break;
   }
   __syncthreads();
@@ -274,7 +284,7 @@ __global__ void prefill_tau_kernel(const float* sample, int64_t n_samp, const in
     const int32_t c = sidx[(int64_t)row * r + k];
     if (c >= 0) { m = fminf(m, sample[(int64_t)row * n_samp + c]); ++have; }
   }
-  tau[row] = (visible <= kCandCap || have == 0 || m == -INFINITY) ? -INFINITY : m;
+  tau[row] = (visible <= kChunkCap || have == 0 || m == -INFINITY) ? -INFINITY : m;
 }
 
 // ------------------------------------------------------------- final select --
@@ -363,8 +373,9 @@ struct PfFinalParams {
   int n_q, H_I, K;
   int64_t T;
   const float* tau;
-  const uint2* cand;
-  const uint32_t* cnt;
+  const uint2* cand;       // [rows][kchunks][kChunkCap]
+  const uint32_t* cnt;     // [rows][kchunks]
+  int kchunks;
   int32_t* idx;            // [B*n_q][K]
 };
 
@@ -409,17 +420,37 @@ __global__ void __launch_bounds__(kPfFinalThreads) prefill_final_kernel(PfFinalP
   const int64_t visible = p.T - p.n_q + t + 1;
   const uint32_t K = (uint32_t)p.K;
   int32_t* out = p.idx + (int64_t)row * p.K;
-  const uint32_t c_all = p.cnt[row];
+  __shared__ uint32_t s_total, s_over;
+  if (tid == 0) {
+    uint32_t tot = 0, over = 0;
+    for (int c = 0; c < p.kchunks; ++c) {
+      const uint32_t n = p.cnt[(int64_t)row * p.kchunks + c];
+      over |= n > (uint32_t)kChunkCap ? 1u : 0u;
+      tot += n;
+    }
+    s_total = tot;
+    s_over = over;
+  }
+  __syncthreads();
+  const uint32_t c_all = s_total;
   const float tau = p.tau[row];
-  const bool fast = c_all <= (uint32_t)kCandCap && (c_all >= K || tau == -INFINITY);
+  const bool fast = !s_over && c_all <= (uint32_t)kCandCap && (c_all >= K || tau == -INFINITY);
 
   uint32_t n_sel = 0;    // selected positions gathered into outp (unsorted)
   if (fast) {
     const uint32_t m = c_all;
-    for (uint32_t i = tid; i < m; i += kPfFinalThreads) {
-      const uint2 v = p.cand[(int64_t)row * kCandCap + i];
-      ck[i] = v.x;
-      cp[i] = v.y;
+    {
+      uint32_t base = 0;
+      for (int c = 0; c < p.kchunks; ++c) {
+        const uint32_t n = p.cnt[(int64_t)row * p.kchunks + c];
+        const uint2* src = p.cand + ((int64_t)row * p.kchunks + c) * kChunkCap;
+        for (uint32_t i = tid; i < n; i += kPfFinalThreads) {
+          const uint2 v = src[i];
+          ck[base + i] = v.x;
+          cp[base + i] = v.y;
+        }
+        base += n;
+      }
     }
     __syncthreads();
     const bool take_all = m <= K;
@@ -554,12 +585,13 @@ static PfWs carve_pf_ws(const csa_index_args* a, void* ws) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   size_t off = 0;
   auto take = [&](size_t n) { uint8_t* p = base ? base + off : nullptr; off += al256p(n); return p; };
-  w.cnt = reinterpret_cast<uint32_t*>(take((size_t)rows * 4));
   w.sample = reinterpret_cast<float*>(take((size_t)rows * n_samp * 4));
   off += select_carve(w.sel, rows, n_samp, base ? base + off : nullptr);
   w.sidx = reinterpret_cast<int32_t*>(take((size_t)rows * pf_sample_r(a->K) * 4));
   w.tau = reinterpret_cast<float*>(take((size_t)rows * 4));
-  w.cand = reinterpret_cast<uint2*>(take((size_t)rows * kCandCap * 8));
+  const int kchunks = (int)((ntiles + kPfChunkTiles - 1) / kPfChunkTiles);
+  w.cnt = reinterpret_cast<uint32_t*>(take((size_t)rows * kchunks * 4));
+  w.cand = reinterpret_cast<uint2*>(take((size_t)rows * kchunks * kChunkCap * 8));
   w.bytes = off;
   return w;
 }
@@ -576,8 +608,6 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   CUtensorMap map;
   if (!make_key_tmap(&map, a->keys, a->T, a->B, a->key_row_stride, a->key_batch_stride))
     return cudaErrorInvalidValue;
-  e = launch_zero(w.cnt, (size_t)rows * 4 + 12, stream);                // counts (rounded to 16 B inside)
-  if (e != cudaSuccess) return e;
   e = launch_zero(w.sel.hist, (size_t)rows * kHistBins * 4, stream);
   if (e != cudaSuccess) return e;
 
@@ -652,6 +682,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   f.tau = w.tau;
   f.cand = w.cand;
   f.cnt = w.cnt;
+  f.kchunks = p.kchunks;
   f.idx = a->idx;
   {
     ProfScope ps(stream, "prefill_final");
