@@ -351,7 +351,7 @@ def run_prefill(args, dev):
     import indexer_selected_sparse_csa2_b200 as csa
     from csa_synth import get_config
     from csa_synth.device import DeviceCase
-    cfg = get_config("prefill_1m")
+    cfg = get_config(args.prefill_config)
     dc = DeviceCase(cfg, device=dev)
     descs = dc.layer_descs(append_rows=True)
     ws = torch.empty(max(csa.csa_layer_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
@@ -381,7 +381,7 @@ def run_prefill(args, dev):
     tflops = flops / (main_ms * 1e-3) / 1e12 if nl else None
     attn_flops = 2.0 * 2.0 * cfg.n_q * cfg.H * cfg.D * (cfg.K + cfg.n_win)
     return {
-        "workload": "prefill_1m", "n_q": cfg.n_q, "T": cfg.T, "K": cfg.K, "W": cfg.W,
+        "workload": cfg.name, "n_q": cfg.n_q, "T": cfg.T, "K": cfg.K, "W": cfg.W,
         "ms_per_chunk": round(ms, 3), "tokens_per_s": round(cfg.n_q / (ms * 1e-3), 1),
         "index_gemm": {"bound": "tensor", "achieved": round(tflops, 1) if tflops else None,
                        "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
@@ -407,6 +407,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--prefill-warmup", type=int, default=1)
+    ap.add_argument("--prefill-config", default="prefill_1m")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -94,6 +94,9 @@ CONFIGS = {
                 LayerSpec(REINDEX, 0, pool_from=0)]),
     "prefill_1m": Config(name="prefill_1m", B=1, T=1 << 20, H=64, H_I=8, K=2048, seed=4,
                          n_q=4096, bf16_latents=True),
+    # a quarter-size prefill chunk (profiling captures that must stay small)
+    "prefill_256k": Config(name="prefill_256k", B=1, T=1 << 18, H=64, H_I=8, K=2048, seed=4,
+                           n_q=1024, bf16_latents=True),
 }
 
 

@@ -3,10 +3,12 @@
 // relu(<qI[t,j], kI[s]>), s <= T - n_q + t; Model techniques map -
 // DeepSeek-V4.1-Flash, "Indexer-selected sparse attention" row).
 //
-// Dense part on the tensor cores: for a block of 32 queries (N = 32 x 8
-// heads = 256 rows of 64 bytes) and 128-position key tiles (M = 128, TMA,
-// 64-byte swizzle), two tcgen05.mma kind::f8f6f4 per tile into a 256-column
-// TMEM accumulator (two of them, double-buffered).  The 1M x 4096 score
+// Dense part on the tensor cores: for a block of 24 queries (N = 24 x 8
+// heads = 192 rows of 64 bytes) and 128-position key tiles (M = 128, TMA,
+// 64-byte swizzle), two tcgen05.mma kind::f8f6f4 per tile into a 192-column
+// TMEM accumulator (two of them, double-buffered).  Twelve epilogue warps
+// (4 TMEM lane quarters x 3 groups of 8 queries) turn the head dots into
+// scores.  The 1M x 4096 score
 // matrix is never stored; selection is exact in three steps:
 //   1  sample pass: the same kernel on every kSampleStride-th key tile writes
 //      those scores; a Top-r select per query gives a threshold tau_t (the
@@ -24,18 +26,18 @@
 
 namespace csa {
 
-constexpr int kPfQPerBlock = 32;                      // queries per N block
-constexpr int kPfN = kPfQPerBlock * 8;                // 256 (8 head rows per query)
+constexpr int kPfQPerBlock = 24;                      // queries per N block
+constexpr int kPfN = kPfQPerBlock * 8;                // 192 (8 head rows per query)
 constexpr int kPfRows = 128;
 constexpr int kPfStages = 8;
 constexpr int kPfStageBytes = kPfRows * 64;
 constexpr int kPfAcc = 2;
-constexpr int kPfEpiWarps = 16;                       // 4 TMEM quarters x 4 query groups of 8
-constexpr int kPfThreads = 64 + 32 * kPfEpiWarps;     // 576
+constexpr int kPfEpiWarps = 12;                       // 4 TMEM quarters x 3 query groups of 8
+constexpr int kPfThreads = 64 + 32 * kPfEpiWarps;     // 448 (register cap 128 per thread)
 constexpr int kSampleStride = 64;                     // sample every 64th key tile
 constexpr int kCandCap = 16384;                       // candidates the final select holds per query
-constexpr int kChunkCap = 8192;                       // candidates kept per (query, key chunk)
-constexpr int kPfChunkTiles = 1024;                   // key tiles per work item
+constexpr int kChunkCapMax = 8192;                    // candidates kept per (query, key chunk), upper bound
+constexpr int kPfChunkTiles = 256;                    // key tiles per work item
 
 static __device__ int g_pf_error;
 
@@ -52,7 +54,8 @@ struct PfParams {
   float* sample;           // [B*n_q][n_samp]    (mode 0)
   int64_t n_samp;
   const float* tau;        // [B*n_q]           (mode 1)
-  uint2* cand;             // [B*n_q][kchunks][kChunkCap] (mode 1): (order key, position)
+  uint2* cand;             // [B*n_q][kchunks][chunk_cap] (mode 1): (order key, position)
+  int chunk_cap;
   uint32_t* cnt;           // [B*n_q][kchunks] hits per (query, key chunk), overflow included
 };
 
@@ -125,6 +128,7 @@ CSA_DEV int64_t pf_tile(const PfParams& p, const PfItem& x, int64_t i) {
   return first + i * kSampleStride;
 }
 
+template <int MODE>   // 0 = sample pass, 1 = main pass (p.mode must match)
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -201,23 +205,28 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
         }
       }
     } else {
-      // epilogue warp e: TMEM quarter e % 4 (32 key rows), query group e / 4 (8 queries)
+      // epilogue warp e: TMEM quarter e % 4 (32 key rows), query group e / 4
+      // (8 queries = 64 accumulator columns, all loaded at once: eight
+      // independent multiply-add chains, packed two heads per instruction)
       const int e = warp - 2;
       const int quarter = warp & 3;
       const int qg = e >> 2;
       const int t0 = x.qb * kPfQPerBlock + qg * 8;          // first query of the group
       const int64_t row0 = (int64_t)x.b * p.n_q + t0;
-      const int64_t lim0 = p.T - p.n_q + t0;                 // last visible position of query t0
+      const int lim0 = (int)(p.T - p.n_q) + t0;              // last visible position of query t0
       const int nlive = min(8, p.n_q - t0);
       float tau[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) tau[k] = (p.mode == 1 && k < nlive) ? p.tau[row0 + k] : 0.f;
-      const float* wq = S.wts + qg * 64;
+      for (int k = 0; k < 8; ++k) tau[k] = (MODE == 1 && k < nlive) ? p.tau[row0 + k] : INFINITY;
+      const float4* wq = reinterpret_cast<const float4*>(S.wts + qg * 64);
       const int kc = (int)(x.kt0 / kPfChunkTiles);
-      for (int64_t i = 0; i < n_t && !failed; ++i) {
-        const int64_t g = run + i;
-        const int a = (int)(g % kPfAcc);
-        if (!mbar_wait(&S.accf[a], (uint32_t)(g / kPfAcc) & 1u, &g_pf_error, kErrWaitAccFull)) { failed = true; break; }
+      uint2* cand_base = p.cand + (row0 * p.kchunks + kc) * (int64_t)p.chunk_cap;
+      const int nt = (int)n_t;
+      const int run32 = (int)(run & 0x7FFFFFFF);
+      for (int i = 0; i < nt; ++i) {
+        const uint32_t g = (uint32_t)(run32 + i);
+        const int a = (int)(g & (kPfAcc - 1));
+        if (!mbar_wait(&S.accf[a], (g / kPfAcc) & 1u, &g_pf_error, kErrWaitAccFull)) { failed = true; break; }
         tc_fence_after();
         const uint32_t col0 = tbase + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(a * kPfN + qg * 64);
         uint32_t r[4][16];
@@ -229,26 +238,44 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.acce[a]);
-        const int64_t tile = pf_tile(p, x, i);
-        const int64_t pos = tile * kPfRows + 32 * quarter + lane;
+        const int tile = MODE == 1 ? (int)x.kt0 + i : (int)pf_tile(p, x, i);
+        const int pos = tile * kPfRows + 32 * quarter + lane;
+        float sc[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float4 wa = *reinterpret_cast<const float4*>(wq + 8 * k);
-          const float4 wb = *reinterpret_cast<const float4*>(wq + 8 * k + 4);
+          const float4 wa = wq[2 * k], wb = wq[2 * k + 1];
           const uint32_t* rr = r[k >> 1] + (k & 1) * 8;
-          const float sc = ((wa.x * fmaxf(__uint_as_float(rr[0]), 0.f) + wa.y * fmaxf(__uint_as_float(rr[1]), 0.f)) +
-                            (wa.z * fmaxf(__uint_as_float(rr[2]), 0.f) + wa.w * fmaxf(__uint_as_float(rr[3]), 0.f))) +
-                           ((wb.x * fmaxf(__uint_as_float(rr[4]), 0.f) + wb.y * fmaxf(__uint_as_float(rr[5]), 0.f)) +
-                            (wb.z * fmaxf(__uint_as_float(rr[6]), 0.f) + wb.w * fmaxf(__uint_as_float(rr[7]), 0.f)));
-          if (k < nlive) {
-            const bool vis = pos <= lim0 + k;
-            if (p.mode == 0) {
-              const int64_t col = (tile / kSampleStride) * kPfRows + 32 * quarter + lane;
-              p.sample[(row0 + k) * p.n_samp + col] = vis ? sc : -INFINITY;
-            } else if (vis && sc >= tau[k]) {
-              const uint32_t slot = atomicAdd(&s_cnt[qg * 8 + k], 1u);
-              if (slot < (uint32_t)kChunkCap)
-                p.cand[((row0 + k) * p.kchunks + kc) * kChunkCap + slot] = make_uint2(order_key(sc), (uint32_t)pos);
+          float2 acc = __fmul2_rn(make_float2(wa.x, wa.y), make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
+                                                                      fmaxf(__uint_as_float(rr[1]), 0.f)));
+          acc = __ffma2_rn(make_float2(wa.z, wa.w),
+                           make_float2(fmaxf(__uint_as_float(rr[2]), 0.f), fmaxf(__uint_as_float(rr[3]), 0.f)), acc);
+          acc = __ffma2_rn(make_float2(wb.x, wb.y),
+                           make_float2(fmaxf(__uint_as_float(rr[4]), 0.f), fmaxf(__uint_as_float(rr[5]), 0.f)), acc);
+          acc = __ffma2_rn(make_float2(wb.z, wb.w),
+                           make_float2(fmaxf(__uint_as_float(rr[6]), 0.f), fmaxf(__uint_as_float(rr[7]), 0.f)), acc);
+          sc[k] = acc.x + acc.y;
+        }
+        // visibility: every position of the tile is visible to every query
+        // of the group unless the tile crosses the causal diagonal
+        const bool all_vis = tile * kPfRows + kPfRows - 1 <= lim0;
+        if (MODE == 0) {
+          const int64_t col = (int64_t)(tile / kSampleStride) * kPfRows + 32 * quarter + lane;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (k < nlive)
+              p.sample[(row0 + k) * p.n_samp + col] = (all_vis || pos <= lim0 + k) ? sc[k] : -INFINITY;
+        } else {
+          bool any = false;                  // tau = +inf for dead queries: never hits
+#pragma unroll
+          for (int k = 0; k < 8; ++k) any |= sc[k] >= tau[k];
+          if (any) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              if (sc[k] >= tau[k] && (all_vis || pos <= lim0 + k)) {
+                const uint32_t slot = atomicAdd(&s_cnt[qg * 8 + k], 1u);
+                if (slot < (uint32_t)p.chunk_cap)
+                  cand_base[(int64_t)k * p.kchunks * p.chunk_cap + slot] = make_uint2(order_key(sc[k]), (uint32_t)pos);
+              }
             }
           }
         }
@@ -257,7 +284,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
     run += n_t;
     if (failed) atomicExch(&any_failed, 1);
     __syncthreads();
-    if (p.mode == 1 && tid < kPfQPerBlock) {
+    if (MODE == 1 && tid < kPfQPerBlock) {
       const int t = x.qb * kPfQPerBlock + tid;
       if (t < p.n_q) p.cnt[((int64_t)x.b * p.n_q + t) * p.kchunks + x.kt0 / kPfChunkTiles] = s_cnt[tid];
     }
@@ -273,7 +300,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
 // tau_t: the smallest of the r best sampled scores, or -inf when every
 // visible position fits in the candidate buffer.
 __global__ void prefill_tau_kernel(const float* sample, int64_t n_samp, const int32_t* sidx, int r, int rows,
-                                   int n_q, int64_t T, float* tau) {
+                                   int n_q, int64_t T, int64_t fit, float* tau) {
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= rows) return;
   const int t = row % n_q;
@@ -284,7 +311,7 @@ __global__ void prefill_tau_kernel(const float* sample, int64_t n_samp, const in
     const int32_t c = sidx[(int64_t)row * r + k];
     if (c >= 0) { m = fminf(m, sample[(int64_t)row * n_samp + c]); ++have; }
   }
-  tau[row] = (visible <= kChunkCap || have == 0 || m == -INFINITY) ? -INFINITY : m;
+  tau[row] = (visible <= fit || have == 0 || m == -INFINITY) ? -INFINITY : m;
 }
 
 // ------------------------------------------------------------- final select --
@@ -373,9 +400,10 @@ struct PfFinalParams {
   int n_q, H_I, K;
   int64_t T;
   const float* tau;
-  const uint2* cand;       // [rows][kchunks][kChunkCap]
+  const uint2* cand;       // [rows][kchunks][chunk_cap]
   const uint32_t* cnt;     // [rows][kchunks]
   int kchunks;
+  int chunk_cap;
   int32_t* idx;            // [B*n_q][K]
 };
 
@@ -425,7 +453,7 @@ __global__ void __launch_bounds__(kPfFinalThreads) prefill_final_kernel(PfFinalP
     uint32_t tot = 0, over = 0;
     for (int c = 0; c < p.kchunks; ++c) {
       const uint32_t n = p.cnt[(int64_t)row * p.kchunks + c];
-      over |= n > (uint32_t)kChunkCap ? 1u : 0u;
+      over |= n > (uint32_t)p.chunk_cap ? 1u : 0u;
       tot += n;
     }
     s_total = tot;
@@ -443,7 +471,7 @@ __global__ void __launch_bounds__(kPfFinalThreads) prefill_final_kernel(PfFinalP
       uint32_t base = 0;
       for (int c = 0; c < p.kchunks; ++c) {
         const uint32_t n = p.cnt[(int64_t)row * p.kchunks + c];
-        const uint2* src = p.cand + ((int64_t)row * p.kchunks + c) * kChunkCap;
+        const uint2* src = p.cand + ((int64_t)row * p.kchunks + c) * p.chunk_cap;
         for (uint32_t i = tid; i < n; i += kPfFinalThreads) {
           const uint2 v = src[i];
           ck[base + i] = v.x;
@@ -577,6 +605,16 @@ static int pf_sample_r(int K) {
   return r < 4 ? 4 : r;
 }
 
+// Candidates kept per (query, key chunk): ~2K are expected per query in
+// total, spread over the chunks; keep a wide margin, at least 2048.
+static int pf_chunk_cap(int64_t ntiles) {
+  const int kchunks = (int)((ntiles + kPfChunkTiles - 1) / kPfChunkTiles);
+  int cap = 16384 / (kchunks > 0 ? kchunks : 1);
+  if (cap < 2048) cap = 2048;
+  if (cap > kChunkCapMax) cap = kChunkCapMax;
+  return cap;
+}
+
 static PfWs carve_pf_ws(const csa_index_args* a, void* ws) {
   PfWs w{};
   const int rows = a->B * a->n_q;
@@ -591,7 +629,7 @@ static PfWs carve_pf_ws(const csa_index_args* a, void* ws) {
   w.tau = reinterpret_cast<float*>(take((size_t)rows * 4));
   const int kchunks = (int)((ntiles + kPfChunkTiles - 1) / kPfChunkTiles);
   w.cnt = reinterpret_cast<uint32_t*>(take((size_t)rows * kchunks * 4));
-  w.cand = reinterpret_cast<uint2*>(take((size_t)rows * kchunks * kChunkCap * 8));
+  w.cand = reinterpret_cast<uint2*>(take((size_t)rows * kchunks * pf_chunk_cap(ntiles) * 8));
   w.bytes = off;
   return w;
 }
@@ -613,7 +651,8 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
 
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(prefill_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmemBytes);
+    cudaFuncSetAttribute(prefill_score_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmemBytes);
+    cudaFuncSetAttribute(prefill_score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmemBytes);
     cudaFuncSetAttribute(prefill_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)((2 * kCandCap + 2 * kPfMaxK) * 4));
     attr = true;
@@ -634,13 +673,14 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   p.tau = w.tau;
   p.cand = w.cand;
   p.cnt = w.cnt;
+  p.chunk_cap = pf_chunk_cap(ntiles);
   const int grid = p.n_items < kNumSMs ? p.n_items : kNumSMs;
 
   // 1. sample pass + per-query threshold
   p.mode = 0;
   {
     ProfScope ps(stream, "prefill_score_tc[sample]");
-    prefill_score_tc_kernel<<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
+    prefill_score_tc_kernel<0><<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
   }
   note_launches(1);
   SelectJob& j = w.sel;
@@ -658,14 +698,18 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   if (e != cudaSuccess) return e;
   {
     ProfScope ps(stream, "prefill_tau");
-    prefill_tau_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(w.sample, n_samp, w.sidx, r, rows, a->n_q, a->T, w.tau);
+    // a query whose visible positions all fit in one key chunk's buffer takes
+    // every position (tau = -inf); with several chunks, each chunk holds its share
+    const int64_t fit = p.kchunks == 1 ? (int64_t)p.chunk_cap : 0;
+    prefill_tau_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(w.sample, n_samp, w.sidx, r, rows, a->n_q, a->T, fit,
+                                                               w.tau);
   }
   note_launches(1);
   // 2. main pass
   p.mode = 1;
   {
     ProfScope ps(stream, "prefill_score_tc[main]");
-    prefill_score_tc_kernel<<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
+    prefill_score_tc_kernel<1><<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
   }
   note_launches(1);
   // 3. exact per-query Top-K
@@ -683,6 +727,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   f.cand = w.cand;
   f.cnt = w.cnt;
   f.kchunks = p.kchunks;
+  f.chunk_cap = p.chunk_cap;
   f.idx = a->idx;
   {
     ProfScope ps(stream, "prefill_final");

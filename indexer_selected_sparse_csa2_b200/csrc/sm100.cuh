@@ -39,11 +39,14 @@ CSA_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}"
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
+// One wait attempt: the thread may sleep (without issuing) until the phase
+// completes or kSuspendNs elapses, so waiting warps do not steal issue slots.
+constexpr uint32_t kSuspendNs = 1000000;   // 1 ms per attempt at most
 CSA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs) : "memory");
   return ok != 0;
 }
 CSA_DEV uint64_t global_ns() {
@@ -51,7 +54,8 @@ CSA_DEV uint64_t global_ns() {
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait for the phase with the given parity; false (and *flag set) on timeout.
+// Bounded wait for the phase with the given parity; false (and *flag set) on
+// timeout (kWaitNs of wall-clock time).
 CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
