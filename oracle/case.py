@@ -20,12 +20,15 @@ from .layers import LayerInputs, run_stack
 class SynthCase:
     """Encoded inputs of one sequence ``b`` of a config (rows built on demand)."""
 
-    def __init__(self, cfg: Config, b: int, sinks: bool = False, threads: int = 4):
+    def __init__(self, cfg: Config, b: int, sinks: bool = False, threads: int = 4,
+                 dense_latents: bool = False):
         self.cfg = cfg
         self.b = b
         self.sinks = sinks
         self.threads = threads
+        self.dense_latents = dense_latents   # hold all fp32 latents of an owner (large caches)
         self._keys = {}
+        self._lat = {}
 
     def keys(self, owner: int) -> np.ndarray:
         if owner not in self._keys:
@@ -34,6 +37,10 @@ class SynthCase:
         return self._keys[owner]
 
     def main_entries(self, owner: int, positions: np.ndarray) -> np.ndarray:
+        if self.dense_latents:
+            if owner not in self._lat:
+                self._lat[owner] = wl.main_latent(self.cfg, owner, self.b, 0, self.cfg.T, threads=self.threads)
+            return fp4_quant_rows(self._lat[owner][np.asarray(positions, dtype=np.int64)])
         return fp4_quant_rows(wl.main_latent_at(self.cfg, owner, self.b, positions))
 
     def main_range(self, owner: int, t0: int, n: int) -> np.ndarray:

@@ -1,0 +1,112 @@
+"""Full-size GPU parity: every workload at its real size, run exactly as the
+benchmark runs it (csa_layer_step over the device-encoded caches, with the
+step's new-token encodes), checked against the oracle on sampled sequences
+(decode) or sampled query tokens (prefill)."""
+import os
+
+import numpy as np
+import pytest
+
+from csa_synth import get_config
+from csa_synth.configs import FULL, REINDEX, REUSE
+from oracle.case import SynthCase
+from oracle import indexer as oi
+from tests.parity import topk_diff, assert_close, check_row_format
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def csa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import indexer_selected_sparse_csa2_b200 as m
+    return m
+
+
+def _compare_layers(cfg, dc, b, res, queries, t_index):
+    """res: oracle results for `queries`; t_index maps query rank -> device row."""
+    n_identical = n_rows = 0
+    for li, L in enumerate(cfg.layers):
+        dl = dc.layers[li]
+        r = res[li]
+        for qr, t in enumerate(queries):
+            n_rows += 1
+            if L.mode == REUSE:
+                src = L.reuse_from
+                g_idx = dc.layers[src].idx[b, t].cpu().numpy()
+                o_idx = r.idx[qr]
+            else:
+                g_idx = dl.idx[b, t].cpu().numpy()
+                o_idx = r.idx[qr]
+                check_row_format(g_idx)
+                if L.mode == REINDEX and L.pool_from >= 0:
+                    P = res[L.pool_from]
+                    S_full = np.full(cfg.T, np.nan)
+                    S_full[P.pool[:P.pool_len].astype(np.int64)] = r.scores[qr]
+                else:
+                    S_full = r.scores[qr]
+                topk_diff(g_idx, o_idx, lambda p: S_full[p])
+                if L.build_pool:
+                    gp = dl.pool[b].cpu().numpy()
+                    gn = int(dl.pool_len[b])
+                    check_row_format(gp)
+                    bm = oi.block_max(r.scores[qr], cfg.pool_block_len)
+                    gblk = np.unique(gp[:gn] // cfg.pool_block_len)
+                    oblk = np.unique(r.pool[:r.pool_len] // cfg.pool_block_len)
+                    pad = lambda a: np.concatenate([a, -np.ones(cfg.pool_blocks - a.size, np.int64)])
+                    topk_diff(pad(gblk), pad(oblk), lambda p: bm[p])
+            if np.array_equal(g_idx, o_idx):
+                n_identical += 1
+                assert_close(dl.out[b, t].cpu().numpy(), r.out[qr], f"layer {li} b {b} t {t} out")
+                assert_close(dl.lse[b, t].cpu().numpy(), r.lse[qr], f"layer {li} b {b} t {t} lse")
+    # near-tie swaps are allowed by the Top-K rule but must stay rare
+    assert n_identical >= 0.75 * n_rows, (n_identical, n_rows)
+
+
+def _run_decode(csa, name, batches):
+    from csa_synth.device import DeviceCase
+    cfg = get_config(name)
+    dc = DeviceCase(cfg, keep_scores=False)
+    csa.csa_layer_step(dc.layer_descs(append_rows=True))
+    torch.cuda.synchronize()
+    assert csa.device_status() == 0
+    for b in batches:
+        case = SynthCase(cfg, b, threads=os.cpu_count() or 4, dense_latents=True)
+        for o in cfg.owners:
+            rows = np.array([0, 1, cfg.T // 2, cfg.T - 1])
+            assert np.array_equal(dc.keys[o][b].cpu().numpy()[rows], case.keys(o)[rows])
+            assert np.array_equal(dc.kv[o][b, torch.from_numpy(rows)].cpu().numpy(), case.main_entries(o, rows))
+        res = case.run(keep_scores=True)
+        _compare_layers(cfg, dc, b, res, [0], None)
+
+
+def test_fullsize_tiny_decode(csa):
+    _run_decode(csa, "tiny_decode", [0])
+
+
+def test_fullsize_decode_64k(csa):
+    _run_decode(csa, "decode_64k", [0, 7])
+
+
+def test_fullsize_stack_128k(csa):
+    _run_decode(csa, "stack_128k", [0, 31])
+
+
+def test_fullsize_hier_1m(csa):
+    _run_decode(csa, "hier_1m", [0, 3])
+
+
+def test_fullsize_prefill_1m(csa):
+    from csa_synth.device import DeviceCase
+    cfg = get_config("prefill_1m")
+    dc = DeviceCase(cfg)
+    csa.csa_layer_step(dc.layer_descs(append_rows=True))
+    torch.cuda.synchronize()
+    assert csa.device_status() == 0
+    qs = [0, 1, 2047, 4095]
+    case = SynthCase(cfg, 0, threads=os.cpu_count() or 4, dense_latents=True)
+    res = case.run(queries=qs, keep_scores=True)
+    _compare_layers(cfg, dc, 0, res, qs, None)
