@@ -22,7 +22,6 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
 import time
 
@@ -74,53 +73,66 @@ def _traffic_record(kernel_src):
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """SM clock and clock-event reasons sampled by NVML every 2 ms during the
+    timed region (read-only queries; no setting is changed)."""
 
-    def __init__(self, index):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "_build", f"clocks_{os.getpid()}.csv")
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.thread = None
+        self.stop_flag = False
+        self.h = None
+        self.err = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+        except Exception as e:  # no NVML: report no clock record
+            self.err = repr(e)
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), get_reasons(self.h)))
+            except Exception as e:
+                self.err = repr(e)
+                return
+            time.sleep(0.002)
 
     def start(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-             "clocks_event_reasons.sw_power_cap")
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.h is None:
+            return
+        import threading
+        self.samples = []
+        self.stop_flag = False
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.h is None or self.thread is None:
+            return {"error": self.err} if self.err else None
+        self.stop_flag = True
+        self.thread.join()
+        if not self.samples:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
 # --------------------------------------------------------------- reference --
@@ -220,26 +232,80 @@ def run_gpu(args, cfg, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    # ---- device-timed steps (L2 flushed between steps, outside the events)
+    # ---- device-timed steps (L2 flushed between steps, outside the events).
+    # The step is captured once into a CUDA graph (as a decode loop runs it);
+    # the library's per-kernel events become graph nodes, read after each replay.
     clocks = Clocks(local_rank)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    csa.profile_enable(True)
+    kernels = {}
+
+    def capture(profile):
+        csa.profile_reset()
+        csa.profile_enable(profile)
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        n_before = csa.launch_count()
+        with torch.cuda.graph(g, stream=cap):
+            csa.csa_layer_step(descs, workspace=ws, stream=cap)
+        torch.cuda.synchronize()
+        csa.profile_enable(False)
+        return g, csa.launch_count() - n_before
+
+    def timed(run, ev_start, ev_end, snap):
+        for i in range(args.steps):
+            flush.zero_()
+            ev_start[i].record(stream)
+            run()
+            ev_end[i].record(stream)
+            if snap:
+                torch.cuda.synchronize()
+                for k, (nl, ms_k) in csa.profile_snapshot().items():
+                    acc = kernels.setdefault(k, [0, 0.0])
+                    acc[0] += nl
+                    acc[1] += ms_k
+        torch.cuda.synchronize()
+
     n0 = csa.launch_count()
+    if args.no_graph:
+        run_step = step
+        launches_per_step = None
+    else:
+        graph, launches_per_step = capture(False)
+        run_step = graph.replay
+        for _ in range(args.warmup):
+            flush.zero_()
+            run_step()
+        torch.cuda.synchronize()
+    # 1. headline: the step with no profiling events
     barrier()
     torch.cuda.synchronize()
     clocks.start()
-    for i in range(args.steps):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize()
+    timed(run_step, starts, ends, False)
     barrier()
     clk = clocks.stop()
-    launches = csa.launch_count() - n0
-    csa.profile_enable(False)
-    kernels = csa.profile_collect()
+    if args.no_graph:
+        launches = csa.launch_count() - n0
+    else:
+        launches = launches_per_step * args.steps
+    # 2. per-kernel breakdown (events around every library kernel, same workload)
+    p_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    p_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if args.no_graph:
+        csa.profile_enable(True)
+        timed(run_step, p_starts, p_ends, False)
+        csa.profile_enable(False)
+        kernels = {k: list(v) for k, v in csa.profile_collect().items()}
+    else:
+        pgraph, _ = capture(True)
+        for _ in range(2):
+            pgraph.replay()
+        torch.cuda.synchronize()
+        timed(pgraph.replay, p_starts, p_ends, True)
+        csa.profile_reset()
+    profiled_ms = sum(s_.elapsed_time(e_) for s_, e_ in zip(p_starts, p_ends)) / args.steps
+    kernels = {k: (int(v[0]), float(v[1])) for k, v in kernels.items()}
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
     t = torch.tensor([ms], dtype=torch.float64, device=dev)
@@ -270,7 +336,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         e_starts[i].record(stream)
         for h, d in h2d_pairs:
             d.copy_(h, non_blocking=True)
-        step()
+        run_step()
         for h, d in d2h_pairs:
             h.copy_(d, non_blocking=True)
         e_ends[i].record(stream)
@@ -310,7 +376,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "fp8/fp4 storage, fp32 scores, fp16 MMA",
         "data": "synthetic (seeded)",
-        "config": {"workload": WORKLOAD, "B_per_gpu": cfg.B, "T": cfg.T, "H": cfg.H, "H_I": cfg.H_I,
+        "config": {"workload": WORKLOAD, "launch": "eager" if args.no_graph else "cuda graph",
+                   "B_per_gpu": cfg.B, "T": cfg.T, "H": cfg.H, "H_I": cfg.H_I,
                    "K": cfg.K, "W": cfg.W, "layers": "Full+pool(2048x8), 3x Reindex-in-pool",
                    "parallelism": f"replicas x{world}", "l2": "flushed between steps (256 MiB write)"},
         "step_hbm_gbs": round(alg / (ms_max * 1e-3) / 1e9, 1),
@@ -329,6 +396,8 @@ def run_gpu(args, cfg, rank, world, local_rank):
             "peak_kind": peak_kind,
         },
         "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / args.steps, 5)} for k, v in kernels.items()},
+        "kernels_note": f"from a second timed pass with an event pair around every kernel "
+                        f"({round(profiled_ms, 4)} ms/step with the events)",
         "gpu_launches": int(launches),
         "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4)},
@@ -398,13 +467,14 @@ def run_prefill(args, dev):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=30.0)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of from a CUDA graph")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--prefill-warmup", type=int, default=1)
     ap.add_argument("--prefill-config", default="prefill_1m")

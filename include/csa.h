@@ -244,6 +244,12 @@ typedef struct {
 } csa_kernel_time;
 int32_t csa_profile_enable(int32_t on);   /* returns the previous state */
 int32_t csa_profile_collect(csa_kernel_time* out, int32_t max_entries);
+/* Launches recorded while a stream was being captured into a CUDA graph
+ * become external event-record nodes, recorded again by every replay:
+ * csa_profile_snapshot() reads the current totals without forgetting the
+ * records (call it after each replay); csa_profile_reset() forgets them. */
+int32_t csa_profile_snapshot(csa_kernel_time* out, int32_t max_entries);
+void csa_profile_reset(void);
 
 /* ------------------------------------------------------------------------ */
 const char* csa_status_string(int32_t status);

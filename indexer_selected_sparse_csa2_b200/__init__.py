@@ -97,12 +97,14 @@ _device_status = _sig("csa_device_status", _i32, [])
 _version = _sig("csa_version", _i32, [])
 _profile_enable = _sig("csa_profile_enable", _i32, [_i32])
 _profile_collect = _sig("csa_profile_collect", _i32, [ctypes.POINTER(KernelTime), _i32])
+_profile_snapshot = _sig("csa_profile_snapshot", _i32, [ctypes.POINTER(KernelTime), _i32])
+_profile_reset = _sig("csa_profile_reset", None, [])
 
 EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
-            "csa_index_noalloc_capacity"]
+            "csa_index_noalloc_capacity", "csa_profile_snapshot", "csa_profile_reset"]
 
 
 def profile_enable(on: bool) -> bool:
@@ -115,6 +117,17 @@ def profile_collect() -> dict:
     buf = (KernelTime * 128)()
     n = _profile_collect(buf, 128)
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 128))}
+
+
+def profile_snapshot() -> dict:
+    """As profile_collect, but keeps the records (graph replays re-record them)."""
+    buf = (KernelTime * 128)()
+    n = _profile_snapshot(buf, 128)
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 128))}
+
+
+def profile_reset() -> None:
+    _profile_reset()
 
 
 class CsaError(RuntimeError):

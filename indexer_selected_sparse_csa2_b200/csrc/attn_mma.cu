@@ -130,6 +130,7 @@ CSA_DEV void dequant_fp8_quarter(const uint8_t* row, int qq, __half* dst) {
 
 template <int H>
 __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnParams p) {
+  pdl_enter();
   constexpr int HB = H / 16;                 // head blocks of 16
   constexpr int EG = 8 / HB;                 // entry groups in phase B
   constexpr int EPW = kTileE / EG;           // entries per warp in phase B
@@ -369,6 +370,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
 // Merge the per-split partial results (log-sum-exp combine): one CTA per
 // (token, head), 128 threads x 4 channels.
 __global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
+  pdl_enter();
   const int bt = blockIdx.x, h = blockIdx.y, H = p.H;
   const int S = p.n_splits;
   __shared__ float wgt_s[64];
@@ -459,12 +461,12 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   dim3 grid(p.n_splits, p.B * p.n_q);
   {
     ProfScope ps(stream, "sparse_attn_mma");
-    sparse_attn_mma_kernel<H><<<grid, kAttnThreads, smem, stream>>>(p);
+    launch_k(sparse_attn_mma_kernel<H>, dim3(grid), dim3(kAttnThreads), smem, stream, p);
   }
   note_launches(1);
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    attn_combine_kernel<<<dim3(p.B * p.n_q, H), 128, 0, stream>>>(p);
+    launch_k(attn_combine_kernel, dim3(dim3(p.B * p.n_q, H)), dim3(128), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <utility>
 
 #include "../../include/csa.h"
 
@@ -82,6 +83,34 @@ CSA_DEV uint4 ld_v4(const void* p) { return *reinterpret_cast<const uint4*>(p); 
 
 }  // namespace csa
 
+// ------------------------------------------- programmatic dependent launch --
+// Every kernel of the library is launched with programmatic stream
+// serialization and starts with pdl_enter(): it lets the next kernel on the
+// stream be scheduled right away (its CTAs then wait in their own
+// pdl_enter()), and waits until the previous kernel on the stream has
+// completed and its writes are visible, before touching any memory.  The
+// launch latency of each kernel thus overlaps the tail of the one before.
+CSA_DEV void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                            Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Host-side launch accounting (see csa_launch_count()) and opt-in event
 // timing of each launch (see csa_profile_enable()).
 namespace csa {
@@ -93,5 +122,6 @@ class ProfScope {
  private:
   cudaStream_t stream_;
   int idx_;
+  bool capturing_ = false;
 };
 }

@@ -55,6 +55,7 @@ constexpr int kRowsPerIter = 16 * kTilesPerIter;       // 64
 constexpr int kRowsPerCtaIter = kRowsPerIter * (kScoreThreads / 32);   // 512
 
 __global__ void __launch_bounds__(kScoreThreads, 2) index_score_decode_kernel(ScoreParams p) {
+  pdl_enter();
   __shared__ uint32_t h[kHistBins];
   __shared__ uint32_t hb[kHistBins];
   const int b = blockIdx.y;
@@ -188,7 +189,7 @@ cudaError_t launch_score_decode(const ScoreParams& p, int B, cudaStream_t stream
   const int nchunks = (int)((p.n + p.chunk - 1) / p.chunk);
   dim3 grid(nchunks > 0 ? nchunks : 1, B);
   ProfScope ps(stream, p.pool ? "index_score_decode[pool]" : "index_score_decode[full]");
-  index_score_decode_kernel<<<grid, kScoreThreads, 0, stream>>>(p);
+  launch_k(index_score_decode_kernel, dim3(grid), dim3(kScoreThreads), 0, stream, p);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -214,12 +215,17 @@ static IndexWs carve_index_ws(const csa_index_args* a, void* ws) {
   const int64_t n = a->pool ? (int64_t)a->pool_cap : a->T;
   uint8_t* base = static_cast<uint8_t*>(ws);
   size_t off = 0;
+  // both first-level histograms side by side, cleared by one launch
+  uint32_t* hists = reinterpret_cast<uint32_t*>(base);
+  off += al256((size_t)2 * B * kHistBins * 4);
   w.scores = reinterpret_cast<float*>(base + off); off += al256((size_t)B * n * 4);
   off += select_carve(w.pos, B, n, base ? base + off : nullptr);
+  w.pos.hist = hists;
   if (a->pool_out) {
     const int64_t nb = (a->T + a->pool_block_len - 1) / a->pool_block_len;
     w.bmax = reinterpret_cast<float*>(base + off); off += al256((size_t)B * nb * 4);
     off += select_carve(w.blk, B, nb, base ? base + off : nullptr);
+    w.blk.hist = hists + (size_t)B * kHistBins;
   }
   w.bytes = off;
   return w;
@@ -239,13 +245,9 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
   const int B = a->B;
   const int64_t n = a->pool ? (int64_t)a->pool_cap : a->T;
   cudaError_t e;
-  // histograms start at zero (pos and block hist are carved first in each job)
-  e = launch_zero(w.pos.hist, (size_t)B * kHistBins * 4, stream);
+  // histograms start at zero (both sit at the start of the workspace)
+  e = launch_zero(w.pos.hist, (size_t)(a->pool_out ? 2 : 1) * B * kHistBins * 4, stream);
   if (e != cudaSuccess) return e;
-  if (a->pool_out) {
-    e = launch_zero(w.blk.hist, (size_t)B * kHistBins * 4, stream);
-    if (e != cudaSuccess) return e;
-  }
   ScoreParams p{};
   p.keys = a->keys;
   p.key_row_stride = a->key_row_stride;

@@ -131,6 +131,7 @@ CSA_DEV int64_t pf_tile(const PfParams& p, const PfItem& x, int64_t i) {
 template <int MODE>   // 0 = sample pass, 1 = main pass (p.mode must match)
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   PfSmem S = carve_pf_smem(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -301,6 +302,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
 // visible position fits in the candidate buffer.
 __global__ void prefill_tau_kernel(const float* sample, int64_t n_samp, const int32_t* sidx, int r, int rows,
                                    int n_q, int64_t T, int64_t fit, float* tau) {
+  pdl_enter();
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= rows) return;
   const int t = row % n_q;
@@ -435,6 +437,7 @@ CSA_DEV float key_score(const uint8_t* krow, const float (*qf)[64], const float 
 }
 
 __global__ void __launch_bounds__(kPfFinalThreads) prefill_final_kernel(PfFinalParams p) {
+  pdl_enter();
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t* ck = reinterpret_cast<uint32_t*>(smem);                 // [kCandCap] keys
   uint32_t* cp = ck + kCandCap;                                      // [kCandCap] positions
@@ -680,7 +683,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   p.mode = 0;
   {
     ProfScope ps(stream, "prefill_score_tc[sample]");
-    prefill_score_tc_kernel<0><<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
+    launch_k(prefill_score_tc_kernel<0>, dim3(grid), dim3(kPfThreads), kPfSmemBytes, stream, map, p);
   }
   note_launches(1);
   SelectJob& j = w.sel;
@@ -701,7 +704,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
     // a query whose visible positions all fit in one key chunk's buffer takes
     // every position (tau = -inf); with several chunks, each chunk holds its share
     const int64_t fit = p.kchunks == 1 ? (int64_t)p.chunk_cap : 0;
-    prefill_tau_kernel<<<(rows + 255) / 256, 256, 0, stream>>>(w.sample, n_samp, w.sidx, r, rows, a->n_q, a->T, fit,
+    launch_k(prefill_tau_kernel, dim3((rows + 255) / 256), dim3(256), 0, stream, w.sample, n_samp, w.sidx, r, rows, a->n_q, a->T, fit,
                                                                w.tau);
   }
   note_launches(1);
@@ -709,7 +712,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   p.mode = 1;
   {
     ProfScope ps(stream, "prefill_score_tc[main]");
-    prefill_score_tc_kernel<1><<<grid, kPfThreads, kPfSmemBytes, stream>>>(map, p);
+    launch_k(prefill_score_tc_kernel<1>, dim3(grid), dim3(kPfThreads), kPfSmemBytes, stream, map, p);
   }
   note_launches(1);
   // 3. exact per-query Top-K
@@ -731,7 +734,7 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   f.idx = a->idx;
   {
     ProfScope ps(stream, "prefill_final");
-    prefill_final_kernel<<<rows, kPfFinalThreads, (2 * kCandCap + 2 * kPfMaxK) * 4, stream>>>(f);
+    launch_k(prefill_final_kernel, dim3(rows), dim3(kPfFinalThreads), (2 * kCandCap + 2 * kPfMaxK) * 4, stream, f);
   }
   note_launches(1);
   return cudaGetLastError();

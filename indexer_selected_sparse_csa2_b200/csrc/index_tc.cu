@@ -78,8 +78,9 @@ CSA_DEV TcSmem carve_tc_smem(uint8_t* raw) {
   return s;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 2)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p) {
+  pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   TcSmem S = carve_tc_smem(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -233,7 +234,9 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
   p.H_I = a->H_I;
   p.T = a->T;
   const int64_t ntiles = (a->T + kTcRows - 1) / kTcRows;
-  int64_t ctas_row = (kNumSMs + a->B - 1) / a->B;
+  // two resident CTAs per SM (about 100 KB of shared memory and 128 TMEM
+  // columns each): twice the loads in flight and epilogue warps per SM
+  int64_t ctas_row = (2 * kNumSMs + a->B - 1) / a->B;
   if (ctas_row > ntiles) ctas_row = ntiles;
   if (ctas_row < 1) ctas_row = 1;
   p.tiles_per_cta = (int)((ntiles + ctas_row - 1) / ctas_row);
@@ -250,7 +253,7 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
     attr = true;
   }
   ProfScope ps(stream, "index_score_tc[full]");
-  index_score_tc_kernel<<<dim3((unsigned)ctas_row, (unsigned)a->B), kTcThreads, kTcSmemBytes, stream>>>(map, p);
+  launch_k(index_score_tc_kernel, dim3(dim3((unsigned)ctas_row, (unsigned)a->B)), dim3(kTcThreads), kTcSmemBytes, stream, map, p);
   note_launches(1);
   return cudaGetLastError();
 }

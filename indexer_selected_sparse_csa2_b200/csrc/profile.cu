@@ -4,7 +4,10 @@
 // before and one just after its kernel; csa_profile_collect() waits for the
 // recorded events and returns, per kernel name, the launch count and the
 // summed event-to-event time.  Disabled by default; enabling it adds two
-// event records per launch to the stream.
+// event records per launch to the stream.  While the stream is being
+// captured into a CUDA graph the records become external event-record nodes,
+// re-recorded by every replay; csa_profile_snapshot() reads them after a
+// replay without forgetting them.
 #include <mutex>
 #include <string>
 #include <vector>
@@ -39,7 +42,11 @@ ProfScope::ProfScope(cudaStream_t s, const char* name) : stream_(s), idx_(-1) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_on) return;
   Rec r{name, take_event(), take_event()};
-  cudaEventRecord(r.start, s);
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &st);
+  capturing_ = st == cudaStreamCaptureStatusActive;
+  if (capturing_) cudaEventRecordWithFlags(r.start, s, cudaEventRecordExternal);
+  else cudaEventRecord(r.start, s);
   g_recs.push_back(r);
   idx_ = (int)g_recs.size() - 1;
 }
@@ -47,7 +54,9 @@ ProfScope::ProfScope(cudaStream_t s, const char* name) : stream_(s), idx_(-1) {
 ProfScope::~ProfScope() {
   if (idx_ < 0) return;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (idx_ < (int)g_recs.size()) cudaEventRecord(g_recs[idx_].stop, stream_);
+  if (idx_ >= (int)g_recs.size()) return;
+  if (capturing_) cudaEventRecordWithFlags(g_recs[idx_].stop, stream_, cudaEventRecordExternal);
+  else cudaEventRecord(g_recs[idx_].stop, stream_);
 }
 
 }  // namespace csa
@@ -63,12 +72,42 @@ int32_t csa_profile_enable(int32_t on) {
   return prev;
 }
 
+static int32_t summarize(std::vector<Rec>& recs, csa_kernel_time* out, int32_t max_entries);
+
+int32_t csa_profile_snapshot(csa_kernel_time* out, int32_t max_entries) {
+  std::vector<Rec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    recs = g_recs;
+  }
+  return summarize(recs, out, max_entries);
+}
+
+void csa_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (Rec& r : g_recs) {
+    g_free.push_back(r.start);
+    g_free.push_back(r.stop);
+  }
+  g_recs.clear();
+}
+
 int32_t csa_profile_collect(csa_kernel_time* out, int32_t max_entries) {
   std::vector<Rec> recs;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     recs.swap(g_recs);
   }
+  const int32_t n = summarize(recs, out, max_entries);
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (Rec& r : recs) {
+    g_free.push_back(r.start);
+    g_free.push_back(r.stop);
+  }
+  return n;
+}
+
+static int32_t summarize(std::vector<Rec>& recs, csa_kernel_time* out, int32_t max_entries) {
   std::vector<std::string> names;
   std::vector<uint64_t> counts;
   std::vector<double> totals;
@@ -85,13 +124,6 @@ int32_t csa_profile_collect(csa_kernel_time* out, int32_t max_entries) {
     }
     counts[k] += 1;
     totals[k] += ms;
-  }
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    for (Rec& r : recs) {
-      g_free.push_back(r.start);
-      g_free.push_back(r.stop);
-    }
   }
   const int32_t n = (int32_t)names.size();
   for (int32_t i = 0; i < n && i < max_entries && out; ++i) {

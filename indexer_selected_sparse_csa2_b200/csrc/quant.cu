@@ -45,6 +45,7 @@ template <int SRC>
 __global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__ src, int64_t n_rows,
                                                         int64_t src_stride_bytes,
                                                         uint8_t* __restrict__ dst, int64_t dst_stride) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
@@ -91,6 +92,7 @@ template <int SRC>
 __global__ void __launch_bounds__(256) quant_fp8w_kernel(const void* __restrict__ src, int64_t n_rows,
                                                          int64_t src_stride_bytes,
                                                          uint8_t* __restrict__ dst, int64_t dst_stride) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
@@ -120,6 +122,7 @@ template <int SRC>
 __global__ void __launch_bounds__(256) quant_plain_kernel(const void* __restrict__ src, int64_t n_rows,
                                                           int dim, int64_t src_stride_bytes,
                                                           uint8_t* __restrict__ dst, int64_t dst_stride) {
+  pdl_enter();
   const int per_row = dim >> 4;
   const int64_t total = n_rows * per_row;
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total;
@@ -155,16 +158,16 @@ cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim
   ProfScope ps(stream, fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? "quant_fp4" : (fmt == CSA_FMT_FP8_E4M3_UE8M0X32 ? "quant_fp8w" : "quant_plain"));
   if (fmt == CSA_FMT_FP4_E2M1_E4M3X16) {
     const int g = grid_for(n_rows, 8);
-    if (src_dtype == CSA_SRC_F32) quant_fp4_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
-    else quant_fp4_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+    if (src_dtype == CSA_SRC_F32) launch_k(quant_fp4_kernel<0>, dim3(g), dim3(256), 0, stream, src, n_rows, sstride, d, dst_row_stride);
+    else launch_k(quant_fp4_kernel<1>, dim3(g), dim3(256), 0, stream, src, n_rows, sstride, d, dst_row_stride);
   } else if (fmt == CSA_FMT_FP8_E4M3_UE8M0X32) {
     const int g = grid_for(n_rows, 8);
-    if (src_dtype == CSA_SRC_F32) quant_fp8w_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
-    else quant_fp8w_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, sstride, d, dst_row_stride);
+    if (src_dtype == CSA_SRC_F32) launch_k(quant_fp8w_kernel<0>, dim3(g), dim3(256), 0, stream, src, n_rows, sstride, d, dst_row_stride);
+    else launch_k(quant_fp8w_kernel<1>, dim3(g), dim3(256), 0, stream, src, n_rows, sstride, d, dst_row_stride);
   } else {
     const int g = grid_for(n_rows * (dim / 16), 256);
-    if (src_dtype == CSA_SRC_F32) quant_plain_kernel<0><<<g, 256, 0, stream>>>(src, n_rows, dim, sstride, d, dst_row_stride);
-    else quant_plain_kernel<1><<<g, 256, 0, stream>>>(src, n_rows, dim, sstride, d, dst_row_stride);
+    if (src_dtype == CSA_SRC_F32) launch_k(quant_plain_kernel<0>, dim3(g), dim3(256), 0, stream, src, n_rows, dim, sstride, d, dst_row_stride);
+    else launch_k(quant_plain_kernel<1>, dim3(g), dim3(256), 0, stream, src, n_rows, dim, sstride, d, dst_row_stride);
   }
   note_launches(1);
   return cudaGetLastError();

@@ -79,6 +79,7 @@ size_t select_carve(SelectJob& j, int B, int64_t n, void* ws) {
 
 // ------------------------------------------------------------------ zero --
 __global__ void zero_kernel(uint4* p, size_t n16) {
+  pdl_enter();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
     p[i] = make_uint4(0, 0, 0, 0);
 }
@@ -89,13 +90,14 @@ cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t stream) {
   int g = (int)((n16 + 255) / 256);
   if (g > kNumSMs * 8) g = kNumSMs * 8;
   ProfScope ps(stream, "zero");
-  zero_kernel<<<g, 256, 0, stream>>>(static_cast<uint4*>(p), n16);
+  launch_k(zero_kernel, dim3(g), dim3(256), 0, stream, static_cast<uint4*>(p), n16);
   note_launches(1);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ hist --
 __global__ void __launch_bounds__(256) select_hist_kernel(SelectJobs jobs) {
+  pdl_enter();
   const SelectJob& J = jobs.j[blockIdx.z];
   const int b = blockIdx.y;
   const int c = blockIdx.x;
@@ -173,6 +175,7 @@ CSA_DEV int threshold_bin(const uint32_t* gh, int K, uint32_t* warp_tot, uint32_
 // candidate buffer, keeping slot order (lane-order prefix via shuffles).
 template <bool VEC>
 __global__ void __launch_bounds__(kExtractThreads) select_extract_kernel(SelectJobs jobs) {
+  pdl_enter();
   const SelectJob& J = jobs.j[blockIdx.z];
   const int b = blockIdx.y;
   if ((int)blockIdx.x * kRunsPerCta >= J.nchunks) return;
@@ -244,6 +247,7 @@ CSA_DEV void write_selected(const SelectJob& J, int b, uint32_t j, int32_t slot)
 }
 
 __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs jobs) {
+  pdl_enter();
   const SelectJob& J = jobs.j[blockIdx.y];
   const int b = blockIdx.x;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -407,13 +411,13 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
   dim3 g(maxc, B, njobs);
   if (build_hist) {
     ProfScope ps(stream, "select_hist");
-    select_hist_kernel<<<g, 256, 0, stream>>>(js);
+    launch_k(select_hist_kernel, dim3(g), dim3(256), 0, stream, js);
     note_launches(1);
   }
   {
     ProfScope ps(stream, "select_extract");
-    if (vec) select_extract_kernel<true><<<g, kExtractThreads, 0, stream>>>(js);
-    else select_extract_kernel<false><<<g, kExtractThreads, 0, stream>>>(js);
+    if (vec) launch_k(select_extract_kernel<true>, dim3(g), dim3(kExtractThreads), 0, stream, js);
+    else launch_k(select_extract_kernel<false>, dim3(g), dim3(kExtractThreads), 0, stream, js);
   }
   const size_t smem = (size_t)kMaxRuns * 4 + (size_t)kListCap * 8;
   static bool attr_set = false;
@@ -423,7 +427,7 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
   }
   {
     ProfScope ps(stream, "select_final");
-    select_final_kernel<<<dim3(B, njobs), kFinalThreads, smem, stream>>>(js);
+    launch_k(select_final_kernel, dim3(dim3(B, njobs)), dim3(kFinalThreads), smem, stream, js);
   }
   note_launches(2);
   return cudaGetLastError();
