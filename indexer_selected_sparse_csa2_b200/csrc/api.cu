@@ -25,6 +25,7 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
 size_t attn_ws_bytes(const csa_attn_args* a);
 int read_tc_error(bool clear);
 int read_pf_error(bool clear);
+int read_at_error(bool clear);
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream);
 
 static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -288,8 +289,8 @@ const char* csa_status_string(int32_t s) {
 }
 
 int32_t csa_device_status(void) {
-  const int a = read_tc_error(true), b = read_pf_error(true);
-  return (int32_t)(a ? a : b);
+  const int a = read_tc_error(true), b = read_pf_error(true), c = read_at_error(true);
+  return (int32_t)(a ? a : (b ? b : c));
 }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

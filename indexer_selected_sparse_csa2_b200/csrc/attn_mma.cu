@@ -22,7 +22,10 @@
 //      so S carries ~22 significant bits of q against the exact fp16 KV;
 //   C  online softmax in the exp2 domain, P stored as fp16;
 //   D  O += P V on tensor cores, O held in registers (fp32).
+#include <cstdlib>
+
 #include "common.cuh"
+#include "attn_tc.cuh"
 
 namespace csa {
 
@@ -472,6 +475,39 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// CSA_ATTN_MMA_SYNC=1 selects the mma.sync kernel for 64 heads too (both
+// kernels are kept: the tcgen05 one is the default).
+static bool use_tc_attention() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("CSA_ATTN_MMA_SYNC");
+    v = (e && e[0] == '1') ? 0 : 1;
+  }
+  return v == 1;
+}
+
+
+// 64 heads run on the tcgen05 kernel; other head counts on the mma.sync kernel.
+static cudaError_t launch_attn_64_tc(AttnParams& p, cudaStream_t stream) {
+  AttnTcParams t;
+  t.B = p.B; t.n_q = p.n_q; t.q = p.q; t.kv = p.kv; t.kv_row_stride = p.kv_row_stride;
+  t.kv_batch_stride = p.kv_batch_stride; t.idx = p.idx; t.K = p.K; t.win = p.win;
+  t.win_row_stride = p.win_row_stride; t.win_batch_stride = p.win_batch_stride; t.n_win = p.n_win;
+  t.scale_log2 = p.scale_log2; t.sink = p.sink; t.out = p.out; t.lse = p.lse; t.n_entries = p.n_entries;
+  // the tcgen05 kernel walks 32-entry tiles: same split boundaries
+  static_assert(kTileE % 32 == 0, "split boundaries must fall on 32-entry tiles");
+  t.tiles_per_split = p.tiles_per_split * (kTileE / 32);
+  t.n_splits = p.n_splits; t.part_o = p.part_o; t.part_ml = p.part_ml;
+  cudaError_t e = launch_attn_tc(t, stream);
+  if (e != cudaSuccess) return e;
+  if (p.n_splits > 1) {
+    ProfScope ps(stream, "attn_combine");
+    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, 64), dim3(128), 0, stream, p);
+    note_launches(1);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream) {
   AttnPlan pl = plan_attn(a);
   AttnParams p{};
@@ -495,7 +531,7 @@ cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t strea
   switch (a->H) {
     case 16: return launch_attn_h<16>(p, stream);
     case 32: return launch_attn_h<32>(p, stream);
-    case 64: return launch_attn_h<64>(p, stream);
+    case 64: return use_tc_attention() ? launch_attn_64_tc(p, stream) : launch_attn_h<64>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -123,7 +123,24 @@ CSA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+CSA_DEV void tmem_ld16f(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
+        "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15])
+      : "r"(taddr));
+}
 CSA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+CSA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+CSA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Named barrier over `count` threads (warps of one role).
+CSA_DEV void named_bar(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
 
 // ------------------------------------------------------------- descriptors --
 // Shared-memory matrix descriptor, K-major, 64-byte swizzle: rows of 64 bytes,
@@ -154,6 +171,27 @@ CSA_DEV uint64_t desc_k_sw128(uint32_t smem_addr) {
 // Instruction descriptor: fp32 accumulate, A/B formats, both K-major, M x N.
 CSA_DEV constexpr uint32_t idesc_make(uint32_t a_fmt, uint32_t b_fmt, int M, int N) {
   return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Same with A MN-major (bit 15); B stays K-major.
+CSA_DEV constexpr uint32_t idesc_make_amn(uint32_t a_fmt, uint32_t b_fmt, int M, int N) {
+  return idesc_make(a_fmt, b_fmt, M, N) | (1u << 15);
+}
+// MN-major, 128-byte swizzle: 64 consecutive MN elements (fp16) per 128-byte
+// row, K rows 128 bytes apart inside an 8-row atom; `lbo` = bytes between
+// 64-element MN blocks, `sbo` = bytes between 8-row K groups.
+CSA_DEV uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Byte offset of (row r, fp16 element c) in 128-byte-swizzled rows of 64
+// fp16 (8-row atoms of 1024 bytes).
+CSA_DEV uint32_t sw128_offset_h(uint32_t r, uint32_t c) {
+  return (r >> 3) * 1024u + (r & 7u) * 128u + ((((c >> 3) ^ r) & 7u) << 4) + (c & 7u) * 2u;
 }
 constexpr uint32_t kFmtE4M3 = 0;   // kind::f8f6f4 operand format
 constexpr uint32_t kFmtF16 = 0;    // kind::f16 operand format

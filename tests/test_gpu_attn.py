@@ -19,7 +19,7 @@ def csa():
     return m
 
 
-def _case(seed, B, n_q, H, T, K, n_win, valid=None, outliers=False, sink=False):
+def _case(seed, B, n_q, H, T, K, n_win, valid=None, outliers=False, sink=False, q_gain=1.0, holes=0.0):
     rng = np.random.default_rng(seed)
     lat = rng.standard_normal((B, T, 512)).astype(np.float32)
     if outliers:
@@ -28,12 +28,14 @@ def _case(seed, B, n_q, H, T, K, n_win, valid=None, outliers=False, sink=False):
     rows = n_q + max(n_win, 1) - 1
     wl = rng.standard_normal((B, rows, 512)).astype(np.float32) * 2
     win = np.stack([oq.fp8_window_quant_rows(wl[b]) for b in range(B)])
-    q = rng.standard_normal((B, n_q, H, 512)).astype(np.float32)
+    q = (rng.standard_normal((B, n_q, H, 512)) * q_gain).astype(np.float32)
     idx = np.full((B, n_q, K), -1, np.int32)
     for b in range(B):
         for t in range(n_q):
             nv = min(K, T) if valid is None else valid
             sel = np.sort(rng.choice(T, size=nv, replace=False)).astype(np.int32)
+            if holes:
+                sel[rng.random(nv) < holes] = -1
             idx[b, t, :nv] = sel
     sk = rng.standard_normal(H).astype(np.float32) if sink else None
     return kv, win, q, idx, sk
@@ -73,6 +75,8 @@ def _oracle(kv, win, q, idx, n_win, scale, sk=None):
     (2, 3, 64, 3000, 64, 16, None),        # several query tokens, sliding window rows
     (1, 1, 64, 50, 0, 1, None),            # window only, single entry
     (1, 1, 16, 300, 1, 0, None),           # a single selected entry, no window
+    (1, 40, 64, 20000, 2048, 128, None),   # prefill-like: 40 tokens, 68 tiles each
+    (1, 2, 64, 3000, 1000, 100, None),     # K and window not multiples of a tile
 ])
 def test_sparse_attention(csa, B, n_q, H, T, K, n_win, valid):
     scale = float(np.float32(1 / np.sqrt(512)))
@@ -110,3 +114,26 @@ def test_dense_equals_full_softmax(csa):
     oo, ol = oa.attend(q[0, 0], X, scale)
     assert_close(go[0, 0], oo, "out")
     assert_close(gl[0, 0], ol, "lse")
+
+
+def test_sharp_scores_and_holes(csa):
+    """Large logits (the running max moves by far more than the lazy-rescale
+    threshold between tiles) and invalid (-1) entries scattered inside tiles."""
+    scale = float(np.float32(1 / np.sqrt(512)))
+    kv, win, q, idx, sk = _case(21, 2, 3, 64, 6000, 1536, 64, q_gain=6.0, holes=0.3, sink=True)
+    go, gl = _gpu(csa, kv, win, q, idx, 64, scale, sk)
+    oo, ol = _oracle(kv, win, q, idx, 64, scale, sk)
+    assert_close(go, oo, "out")
+    assert_close(gl, ol, "lse")
+
+
+def test_mma_sync_kernel_for_64_heads(csa):
+    """The mma.sync kernel that 64 heads run on when CSA_ATTN_MMA_SYNC=1 (the
+    tcgen05 kernel is the default) passes the same cases."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, CSA_ATTN_MMA_SYNC="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k", "not mma_sync_kernel"],
+                       env=env, capture_output=True, text=True, cwd=os.path.dirname(os.path.dirname(__file__)))
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
