@@ -494,9 +494,9 @@ static cudaError_t launch_attn_64_tc(AttnParams& p, cudaStream_t stream) {
   t.kv_batch_stride = p.kv_batch_stride; t.idx = p.idx; t.K = p.K; t.win = p.win;
   t.win_row_stride = p.win_row_stride; t.win_batch_stride = p.win_batch_stride; t.n_win = p.n_win;
   t.scale_log2 = p.scale_log2; t.sink = p.sink; t.out = p.out; t.lse = p.lse; t.n_entries = p.n_entries;
-  // the tcgen05 kernel walks 32-entry tiles: same split boundaries
-  static_assert(kTileE % 32 == 0, "split boundaries must fall on 32-entry tiles");
-  t.tiles_per_split = p.tiles_per_split * (kTileE / 32);
+  // the tcgen05 kernel walks 64-entry tiles: same split boundaries
+  static_assert(kTileE == 64, "split boundaries must fall on 64-entry tiles");
+  t.tiles_per_split = p.tiles_per_split;
   t.n_splits = p.n_splits; t.part_o = p.part_o; t.part_ml = p.part_ml;
   cudaError_t e = launch_attn_tc(t, stream);
   if (e != cudaSuccess) return e;

@@ -5,27 +5,34 @@
 // entries plus the FP8 window, K = V = the 512-wide latent; Model techniques
 // map - DeepSeek-V4.1-Flash, "Multi-head latent attention", "Indexer-selected
 // sparse attention", "Sliding-window attention" and "Learnable attention
-// sink" rows).  Per 32-entry tile of one token:
+// sink" rows).  Per 64-entry tile of one token:
 //   S2 = Q2 K^T   tcgen05.mma kind::f16, M = 128 rows of Q2: row 2h is the
 //                 fp16 hi part of head h's query, row 2h+1 the lo part
-//                 fp16(q - hi); N = 32 entries, K = 512; fp32 in TMEM.  The
-//                 softmax adds the two rows of a head (neighbouring lanes of
-//                 one warp), which carries ~22 bits of q against the exactly
-//                 dequantised fp16 entries.
+//                 fp16(q - hi); N = 64 entries, K = 512; fp32 in TMEM.  The
+//                 first 384 channels of Q2 stay in TMEM as the A operand
+//                 (no shared-memory traffic for them), the last 128 in
+//                 shared memory.  The softmax adds the two rows of a head
+//                 (neighbouring lanes of one warp), which carries ~22 bits of
+//                 q against the exactly dequantised fp16 entries.
 //   O^T += V^T P^T  tcgen05.mma kind::f16, M = 128 latent channels (4
-//                 chunks), N = 64 heads, K = 32 entries, fp32 in TMEM.  The
+//                 chunks), N = 64 heads, K = 64 entries, fp32 in TMEM, once
+//                 for the fp16 hi part of P and once for the lo part.  The
 //                 same shared-memory tile of dequantised entries is the
 //                 K-major B operand of S2 and the MN-major A operand here.
 // Warp roles: warps 0-3 softmax / output (one TMEM lane quarter each; the
-// two lanes of a head split the tile's entries), warps 4-7 gather +
-// dequantise (8 threads per 8 entries and 128 channels; the next tile's raw
-// bytes are loaded into registers while the current one is decoded), warp 8
-// issues the S2 MMAs, warp 9 the PV MMAs.  The entry tile, P and S are
-// double buffered, so tile i+1 is dequantised and its S2 computed while the
+// two lanes of a head split the tile's entries), warps 4-11 gather +
+// dequantise (8 lanes take 8 entries, 4 lanes per entry, 128 channels each;
+// the next tile's raw bytes are loaded into registers while the current one
+// is decoded), warp 12 issues the S2 MMAs, warp 13 the PV MMAs.  Entry
+// tiles and P are double buffered, so tile i+1 is dequantised while S2, the
 // softmax and PV of tile i run.  Online softmax in the exp2 domain with lazy
 // rescaling: the running max only moves when a tile's max exceeds it by more
 // than 8, and only then are the O^T accumulators rescaled in TMEM.
 //
+// Channel order: inside every group of 8 channels the staged operands hold
+// channels (0, 4, 1, 5, 2, 6, 3, 7), so one 32-bit word of FP4 codes turns
+// into four fp16 pairs with shifts and masks only.  Q2 uses the same order
+// (the dot products are unchanged) and the output un-permutes O^T's rows.
 // Main (FP4) entries are staged as E2M1 * s * 2^-7 (exact in fp16, one
 // multiply per channel pair); their logits are scaled by 2^7 and their
 // probabilities by 2^7 in P, which leaves S and O unchanged.  Window entries
@@ -35,18 +42,23 @@
 
 namespace csa {
 
-
 constexpr int kAtH = 64;                  // heads
-constexpr int kAtE = 32;                  // entries per tile
-constexpr int kAtThreads = 320;           // 10 warps
-constexpr int kAtQBytes = 128 * 512 * 2;  // Q2: 128 rows x 512 fp16
-constexpr int kAtKVBytes = kAtE * 512 * 2;        // one entry tile (8 blocks of 64 channels)
-constexpr int kAtKVBlk = kAtE * 128;              // bytes of one 64-channel block
-constexpr int kAtPBytes = kAtH * kAtE * 2;        // one P^T tile: 64 head rows x 64 B
-constexpr int kAtXSBytes = kAtE * kAtH * 4;
-constexpr size_t kAtSmemBytes = 1024 + kAtQBytes + 2 * kAtKVBytes + 2 * kAtPBytes + kAtXSBytes + 1024;
-constexpr uint32_t kAtTmemCols = 512;     // S buffers: cols 0..31, 32..63; O^T chunk c: cols 64 + 64c
-constexpr uint32_t kAtOCol = 64;
+constexpr int kAtE = 64;                  // entries per tile
+constexpr int kAtDeqWarps = 8;
+constexpr int kAtWarpS = 4 + kAtDeqWarps;           // S2 issuer
+constexpr int kAtWarpPV = kAtWarpS + 1;             // PV issuer
+constexpr int kAtThreads = 32 * (kAtWarpPV + 1);    // 448
+constexpr int kAtQTmemBlocks = 6;                   // 64-channel blocks of Q2 in TMEM
+constexpr int kAtQSmemBlocks = 8 - kAtQTmemBlocks;  // ... and in shared memory
+constexpr int kAtQBlkBytes = 128 * 128;             // 128 rows x 64 fp16
+constexpr int kAtKVBlk = kAtE * 128;                // one 64-channel block of an entry tile
+constexpr int kAtKVBytes = 8 * kAtKVBlk;            // 64 KB
+constexpr int kAtPBytes = kAtH * kAtE * 2;          // P^T part (hi or lo): 64 head rows x 128 B
+constexpr size_t kAtSmemBytes = 1024 + (size_t)kAtQSmemBlocks * kAtQBlkBytes + 2 * kAtKVBytes + 4 * kAtPBytes + 1024;
+constexpr uint32_t kAtTmemCols = 512;
+constexpr uint32_t kAtSCol = 32 * kAtQTmemBlocks;   // S2: 64 fp32 columns after Q2
+constexpr uint32_t kAtOCol = 256;                   // O^T chunk c: columns 256 + 64c
+static_assert(kAtSCol + kAtE <= kAtOCol, "TMEM map");
 constexpr float kAtLog2e = 1.4426950408889634f;
 constexpr float kAtLn2 = 0.6931471805599453f;
 constexpr float kAtRescale = 8.0f;        // lazy-rescale threshold (exp2 units)
@@ -54,12 +66,11 @@ constexpr float kAtRescale = 8.0f;        // lazy-rescale threshold (exp2 units)
 static __device__ int g_at_error;
 
 struct AtSmem {
-  uint8_t* q2;
-  uint8_t* kv;      // 2 buffers
-  uint8_t* p;       // 2 buffers
-  float* xs;        // [entry][head] lo-part logits
+  uint8_t* q2;      // Q2 channels 384..511 (2 blocks)
+  uint8_t* kv;      // 2 entry tiles
+  uint8_t* p;       // 2 x (P^T hi, P^T lo)
   float* scl;       // [64] per-head output scale
-  float* alpha_s;   // [64]
+  float* alpha_s;   // [2][64] by tile parity (a warp may run one tile ahead)
   uint64_t* bars;
   uint32_t* tmem_base;
 };
@@ -68,12 +79,11 @@ CSA_DEV AtSmem carve_at(uint8_t* raw) {
   AtSmem s;
   uintptr_t base = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~(uintptr_t)1023;
   uint8_t* p = reinterpret_cast<uint8_t*>(base);
-  s.q2 = p; p += kAtQBytes;
+  s.q2 = p; p += kAtQSmemBlocks * kAtQBlkBytes;
   s.kv = p; p += 2 * kAtKVBytes;
-  s.p = p; p += 2 * kAtPBytes;
-  s.xs = reinterpret_cast<float*>(p); p += kAtXSBytes;
+  s.p = p; p += 4 * kAtPBytes;
   s.scl = reinterpret_cast<float*>(p); p += 64 * 4;
-  s.alpha_s = reinterpret_cast<float*>(p); p += 64 * 4;
+  s.alpha_s = reinterpret_cast<float*>(p); p += 2 * 64 * 4;
   s.bars = reinterpret_cast<uint64_t*>(p); p += 16 * 8;
   s.tmem_base = reinterpret_cast<uint32_t*>(p);
   return s;
@@ -82,25 +92,47 @@ CSA_DEV AtSmem carve_at(uint8_t* raw) {
 CSA_DEV uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 CSA_DEV __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// Channel held at position p (0..7) of an 8-channel group.
+CSA_DEV int perm8(int p) { return (p >> 1) + 4 * (p & 1); }
+
 // Integer-pipe decoders (the conversion pipe is the scarce one here).
-// A 4-bit E2M1 code n placed at bits 0-3 (and 16-19) becomes the fp16 value
-// E2M1(n) * 2^-14 by moving its magnitude bits to fp16 bits 9-11 and its sign
-// to bit 15: E2M1's exponent field lines up with the low fp16 exponent bits
-// and its subnormal (0.5) with the fp16 subnormal 2^-15.
-CSA_DEV uint32_t e2m1x2_bits_m14(uint32_t t) {
-  return ((t << 9) & 0x0E000E00u) | ((t << 12) & 0x80008000u);
-}
 // An 8-bit E4M3 code c at bits 0-7 (and 16-23) becomes the fp16 value
-// E4M3(c) * 2^-8 the same way (exponent and mantissa shifted by 7, sign to
-// bit 15); E4M3 subnormals land on fp16 subnormals, so every code is exact.
+// E4M3(c) * 2^-8 by moving exponent and mantissa up by 7 and the sign to bit
+// 15; E4M3 subnormals land on fp16 subnormals, so every code is exact.  Bits
+// 8-15 and 24-31 of t are ignored.
 CSA_DEV uint32_t e4m3x2_bits_m8(uint32_t t) {
   return ((t << 7) & 0x3F803F80u) | ((t << 8) & 0x80008000u);
+}
+// The FP4 codes of channels kk and kk+4 of a word of 8 codes (channel c in
+// bits 4c..4c+3) as fp16 E2M1 * 2^-14: the E2M1 magnitude bits go to fp16
+// bits 9-11 (its exponent field lines up with the low fp16 exponent bits and
+// its subnormal 0.5 with the fp16 subnormal 2^-15), the sign to bit 15.
+template <int kk>
+CSA_DEV uint32_t e2m1_pair_m14(uint32_t w) {
+  const uint32_t mag = kk < 3 ? (w << (9 - 4 * kk)) : (w >> 3);
+  const uint32_t sgn = w << (12 - 4 * kk);
+  return (mag & 0x0E000E00u) | (sgn & 0x80008000u);
 }
 constexpr uint32_t kH2Exp15 = 0x78007800u;   // fp16x2 {2^15, 2^15}
 CSA_DEV float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// fp16 hi / lo parts of 8 channels (a: channels 0-3, c: 4-7) in the staged
+// order, as four packed pairs.
+CSA_DEV void q_hilo_perm8(float4 a, float4 c, bool lo, uint32_t (&o)[4]) {
+  const float f0[4] = {a.x, a.y, a.z, a.w}, f1[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 hi = __floats2half2_rn(f0[k], f1[k]);       // channels k, k + 4
+    if (!lo) {
+      o[k] = h2u(hi);
+    } else {
+      const float2 hf = __half22float2(hi);
+      o[k] = h2u(__floats2half2_rn(f0[k] - hf.x, f1[k] - hf.y));
+    }
+  }
 }
 
 // Bounded wait taken by a whole warp; the result is the same in every lane, so
@@ -113,13 +145,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   pdl_enter();
   extern __shared__ uint8_t smem_raw[];
   AtSmem S = carve_at(smem_raw);
-  uint64_t* kv_full = S.bars + 0;    // [2] dequant -> MMA (4 warp arrivals)
+  uint64_t* kv_full = S.bars + 0;    // [2] dequant -> S2 issuer (8 warp arrivals)
   uint64_t* kv_free = S.bars + 2;    // [2] PV done: entry tile and P buffer reusable
-  uint64_t* s_full = S.bars + 4;     // [2] S2 in TMEM
-  uint64_t* s_free = S.bars + 6;     // [2] S2 read by the softmax (4 warp arrivals)
-  uint64_t* p_full = S.bars + 8;     // [2] P written, O^T rescaled (4 warp arrivals)
-  uint64_t* o_done = S.bars + 10;    // one phase per PV
-  uint64_t* drain = S.bars + 11;     // [2] all MMAs of an issuer retired (teardown)
+  uint64_t* s_full = S.bars + 4;     // S2 in TMEM
+  uint64_t* s_free = S.bars + 5;     // S2 read by the softmax (4 warp arrivals)
+  uint64_t* p_full = S.bars + 6;     // [2] P written, O^T rescaled (4 warp arrivals)
+  uint64_t* o_done = S.bars + 8;     // one phase per PV
+  uint64_t* drain = S.bars + 9;      // [2] all MMAs of an issuer retired (teardown)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bt = blockIdx.y;
   const int b = bt / p.n_q, tq = bt - b * p.n_q;
@@ -131,17 +163,17 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
 
   if (tid == 0) {
     for (int k = 0; k < 2; ++k) {
-      mbar_init(kv_full + k, 4);
+      mbar_init(kv_full + k, kAtDeqWarps);
       mbar_init(kv_free + k, 1);
-      mbar_init(s_full + k, 1);
-      mbar_init(s_free + k, 4);
       mbar_init(p_full + k, 4);
+      mbar_init(drain + k, 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
     mbar_init(o_done, 1);
-    mbar_init(drain, 1);
-    mbar_init(drain + 1, 1);
     fence_mbar_init();
   }
+
   // gather role: 8 consecutive lanes take 8 different entries, so each
   // quarter-warp phase of a 16-byte shared store covers all 32 banks
   const int jd = tid - 128;
@@ -172,63 +204,85 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }                                                                                          \
   } while (0)
   // the first tile's entries are in flight while q is staged
-  if (warp >= 4 && warp < 8 && nt > 0) CSA_AT_FETCH(tile0);
-  // Q2 rows (2h, 2h+1) = (hi, lo) of head h, fp16, K-major 128-byte swizzle,
-  // 8 blocks of 64 channels
-  {
-    const float* qg = p.q + (int64_t)bt * kAtH * kD;
-#pragma unroll 2
-    for (int i = tid; i < kAtH * (kD / 8); i += kAtThreads) {
-      const int h = i / (kD / 8), c8 = i % (kD / 8);        // 8 channels at 8*c8
-      const float4 a = reinterpret_cast<const float4*>(qg + (int64_t)h * kD + 8 * c8)[0];
-      const float4 c = reinterpret_cast<const float4*>(qg + (int64_t)h * kD + 8 * c8)[1];
-      const float f[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __half2 hh = __floats2half2_rn(f[2 * k], f[2 * k + 1]);
-        const float2 hf = __half22float2(hh);
-        hi[k] = h2u(hh);
-        lo[k] = h2u(__floats2half2_rn(f[2 * k] - hf.x, f[2 * k + 1] - hf.y));
-      }
-      const int d = 8 * c8;
-      const uint32_t blk = (uint32_t)(d >> 6) * (128 * 128);
-      *reinterpret_cast<uint4*>(S.q2 + blk + sw128_offset_h(2 * h, d & 63)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(S.q2 + blk + sw128_offset_h(2 * h + 1, d & 63)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-  }
-  fence_proxy_async_smem();
-  if (warp == 8) tmem_alloc(S.tmem_base, kAtTmemCols);
+  const bool is_deq = warp >= 4 && warp < kAtWarpS;
+  if (is_deq && nt > 0) CSA_AT_FETCH(tile0);
+
+  if (warp == kAtWarpS) tmem_alloc(S.tmem_base, kAtTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *S.tmem_base;
 
-  if (warp == 8) {
+  // ---- Q2 staging.  TMEM part (channels 0..383): TMEM column j of row
+  // r = 2h + part holds the pair of channels (8g + (j & 3), 8g + (j & 3) + 4),
+  // g = j / 4; lane quarter qq is written by warps qq, qq + 4 and qq + 8, four
+  // 16-column stores each.
+  const float* qg = p.q + (int64_t)bt * kAtH * kD;
+  if (warp < kAtWarpS) {
+    const int qq = warp & 3, wr = warp >> 2;
+    const int r = 32 * qq + lane, h = r >> 1;
+    const bool lo = r & 1;
+    const float4* qrow = reinterpret_cast<const float4*>(qg + (int64_t)h * kD);
+#pragma unroll 1
+    for (int u = 4 * wr; u < 4 * wr + 4; ++u) {         // columns 16u .. 16u + 15 = channels 32u .. 32u + 31
+      float4 f[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) f[k] = qrow[8 * u + k];
+      uint32_t v[16];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t o[4];
+        q_hilo_perm8(f[2 * g], f[2 * g + 1], lo, o);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[4 * g + k] = o[k];
+      }
+      tmem_st16(tbase + ((uint32_t)(32 * qq) << 16) + 16u * u, v);
+    }
+    tmem_wait_st();
+  }
+  // shared part (channels 384..511): two K-major 128-byte-swizzled blocks
+  for (int i = tid; i < 128 * 16; i += kAtThreads) {
+    const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
+    const int h = r >> 1;
+    const float4* src = reinterpret_cast<const float4*>(qg + (int64_t)h * kD + 384 + 64 * kb + 8 * c8);
+    uint32_t o[4];
+    q_hilo_perm8(src[0], src[1], r & 1, o);
+    *reinterpret_cast<uint4*>(S.q2 + kb * kAtQBlkBytes + sw128_offset_h(r, 8 * c8)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  if (warp == kAtWarpS) {
     // ------------------------------------------------------------ S2 issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_make(kFmtF16, kFmtF16, 128, kAtE);
       const uint32_t q2a = smem_u32(S.q2), kva = smem_u32(S.kv);
       for (int t = 0; t < nt; ++t) {
-        const int bi = t & 1, ui = t >> 1;
-        if (!mbar_wait(kv_full + bi, (uint32_t)ui & 1u, &g_at_error, kErrWaitTmaFull)) break;
-        if (t >= 2 && !mbar_wait(s_free + bi, (uint32_t)(ui - 1) & 1u, &g_at_error, kErrWaitAccEmpty)) break;
+        const int bi = t & 1;
+        if (!mbar_wait(kv_full + bi, (uint32_t)(t >> 1) & 1u, &g_at_error, kErrWaitTmaFull)) break;
+        if (t >= 1 && !mbar_wait(s_free, (uint32_t)(t - 1) & 1u, &g_at_error, kErrWaitAccEmpty)) break;
         tc_fence_after();
-        const uint32_t kvb = kva + (uint32_t)bi * kAtKVBytes;
-#pragma unroll 4
+        const uint32_t kvt = kva + (uint32_t)bi * kAtKVBytes;
+#pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t kb = ks >> 2, sub = ks & 3;
-          const uint64_t ad = desc_k_sw128(q2a + kb * (128 * 128) + sub * 32);
-          const uint64_t bd = desc_k_sw128(kvb + kb * kAtKVBlk + sub * 32);
-          mma_f16_ss(tbase + 32u * bi, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+          const uint64_t bd = desc_k_sw128(kvt + kb * kAtKVBlk + sub * 32);
+          if (kb < (uint32_t)kAtQTmemBlocks) {
+            mma_f16_ts(tbase + kAtSCol, tbase + kb * 32 + sub * 8, bd, idesc_s, ks > 0 ? 1u : 0u);
+          } else {
+            const uint64_t ad = desc_k_sw128(q2a + (kb - kAtQTmemBlocks) * kAtQBlkBytes + sub * 32);
+            mma_f16_ss(tbase + kAtSCol, ad, bd, idesc_s, 1u);
+          }
         }
-        mma_commit(s_full + bi);
+        mma_commit(s_full);
       }
       // every issued MMA has retired before the accumulators are released
       mma_commit(drain);
       mbar_wait(drain, 0u, &g_at_error, kErrWaitAccFull);
     }
-  } else if (warp == 9) {
+  } else if (warp == kAtWarpPV) {
     // ------------------------------------------------------------ PV issuer
     if (lane == 0) {
       constexpr uint32_t idesc_o = idesc_make_amn(kFmtF16, kFmtF16, 128, kAtH);
@@ -237,16 +291,18 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
         const int bi = i & 1;
         if (!mbar_wait(p_full + bi, (uint32_t)(i >> 1) & 1u, &g_at_error, kErrWaitAccFull)) break;
         tc_fence_after();
-        const uint32_t kvb = kva + (uint32_t)bi * kAtKVBytes, pb = pa + (uint32_t)bi * kAtPBytes;
+        const uint32_t kvt = kva + (uint32_t)bi * kAtKVBytes, pb = pa + (uint32_t)bi * 2 * kAtPBytes;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
           for (int ks = 0; ks < kAtE / 16; ++ks) {
-            // A = V^T: channels 128c.. (two 64-channel blocks), entries 16ks..
-            const uint64_t ad = desc_mn_sw128(kvb + (uint32_t)(2 * c) * kAtKVBlk + (uint32_t)ks * 2048, kAtKVBlk, 1024);
-            // B = P^T: 64 head rows of 32 entries (64-byte swizzle), entries 16ks..
-            const uint64_t bd = desc_k_sw64(pb + (uint32_t)ks * 32);
-            mma_f16_ss(tbase + kAtOCol + 64u * c, ad, bd, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
+            // A = V^T: positions 128c.. (two 64-position blocks), entries 16ks..
+            const uint64_t ad = desc_mn_sw128(kvt + (uint32_t)(2 * c) * kAtKVBlk + (uint32_t)ks * 2048, kAtKVBlk, 1024);
+            // B = P^T hi, then lo: 64 head rows of 64 entries (128-byte swizzle), entries 16ks..
+            const uint64_t bh = desc_k_sw128(pb + (uint32_t)ks * 32);
+            const uint64_t bl = desc_k_sw128(pb + kAtPBytes + (uint32_t)ks * 32);
+            mma_f16_ss(tbase + kAtOCol + 64u * c, ad, bh, idesc_o, (i > 0 || ks > 0) ? 1u : 0u);
+            mma_f16_ss(tbase + kAtOCol + 64u * c, ad, bl, idesc_o, 1u);
           }
         }
         mma_commit(kv_free + bi);
@@ -255,74 +311,61 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       mma_commit(drain + 1);
       mbar_wait(drain + 1, 0u, &g_at_error, kErrWaitAccFull);
     }
-  } else if (warp >= 4) {
+  } else if (is_deq) {
     // --------------------------------------------------- gather + dequantise
     for (int i = 0; i < nt; ++i) {
       const int bi = i & 1;
       if (i >= 2 && !mbar_wait_warp(kv_free + bi, (uint32_t)((i >> 1) - 1) & 1u, kErrWaitSmemEmpty)) break;
       uint8_t* kt = S.kv + bi * kAtKVBytes;
-      // channels [128*q4, 128*q4 + 128) of entry e -> fp16 at (e, d)
+      // channels [128*q4, 128*q4 + 128) of entry e, one 16-byte chunk (8
+      // positions) per group of 8 channels
       if (kind == 1) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {                 // 16 code bytes = 32 channels = 2 scale blocks
-          const uint32_t cw[4] = {rr[k].x, rr[k].y, rr[k].z, rr[k].w};
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            // block scale s as fp16 s * 2^7 (exact: s <= 448 < 2^9)
-            const int sb = 2 * k + half;
-            uint32_t sc = ((sb < 4 ? rex.x : rex.y) >> (8 * (sb & 3))) & 0xFFu;
-            sc |= sc << 16;
-            const __half2 s2 = __hmul2(u2h(e4m3x2_bits_m8(sc)), u2h(kH2Exp15));
-#pragma unroll
-            for (int wi = 0; wi < 2; ++wi) {           // one word = 8 channels
-              const uint32_t w = cw[2 * half + wi];
-              const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-              uint32_t o[4];
-#pragma unroll
-              for (int bb = 0; bb < 4; ++bb) {
-                // channels 2bb, 2bb+1 of the word: low nibble -> low half
-                const uint32_t t = __byte_perm(lo, hi, bb | (bb << 4) | ((4 + bb) << 8) | ((4 + bb) << 12));
-                // (E2M1 * 2^-14) * (s * 2^7) = E2M1 * s * 2^-7: at most 6
-                // significant bits and >= 2^-17, so exact in fp16
-                o[bb] = h2u(__hmul2(u2h(e2m1x2_bits_m14(t)), s2));
-              }
-              const int d = 128 * q4 + 32 * k + 16 * half + 8 * wi;
-              *reinterpret_cast<uint4*>(kt + (uint32_t)(d >> 6) * kAtKVBlk + sw128_offset_h(e, d & 63)) =
-                  make_uint4(o[0], o[1], o[2], o[3]);
-            }
-          }
+        for (int wq = 0; wq < 16; ++wq) {
+          const uint4 r4 = rr[wq >> 2];
+          const uint32_t w = (wq & 3) == 0 ? r4.x : (wq & 3) == 1 ? r4.y : (wq & 3) == 2 ? r4.z : r4.w;
+          // block scale s (16 channels) as fp16 s * 2^7 (exact: s <= 448 < 2^9)
+          const int sb = wq >> 1;
+          uint32_t sc = ((sb < 4 ? rex.x : rex.y) >> (8 * (sb & 3))) & 0xFFu;
+          sc |= sc << 16;
+          const __half2 s2 = __hmul2(u2h(e4m3x2_bits_m8(sc)), u2h(kH2Exp15));
+          // (E2M1 * 2^-14) * (s * 2^7) = E2M1 * s * 2^-7: at most 6
+          // significant bits and >= 2^-17, so exact in fp16
+          const uint32_t o0 = h2u(__hmul2(u2h(e2m1_pair_m14<0>(w)), s2));
+          const uint32_t o1 = h2u(__hmul2(u2h(e2m1_pair_m14<1>(w)), s2));
+          const uint32_t o2 = h2u(__hmul2(u2h(e2m1_pair_m14<2>(w)), s2));
+          const uint32_t o3 = h2u(__hmul2(u2h(e2m1_pair_m14<3>(w)), s2));
+          const int d = 128 * q4 + 8 * wq;
+          *reinterpret_cast<uint4*>(kt + (uint32_t)(d >> 6) * kAtKVBlk + sw128_offset_h(e, d & 63)) =
+              make_uint4(o0, o1, o2, o3);
         }
       } else if (kind == 2) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {                 // 16 code bytes = 16 channels
-          const int ex = (int)((rex.x >> (8 * (k >> 1))) & 0xFF);   // UE8M0: scale 2^(ex - 127)
-          const uint32_t cw[4] = {rr[k].x, rr[k].y, rr[k].z, rr[k].w};
-          uint32_t o[8];
+        for (int g = 0; g < 16; ++g) {                // 8 code bytes = 8 channels
+          const uint4 r4 = rr[g >> 1];
+          const uint32_t w0 = (g & 1) ? r4.z : r4.x, w1 = (g & 1) ? r4.w : r4.y;   // channels 0-3, 4-7
+          const int ex = (int)((rex.x >> (8 * (g >> 2))) & 0xFF);   // UE8M0: scale 2^(ex - 127)
+          uint32_t o[4];
           if (ex >= 105 && ex <= 134) {
             // E4M3 * 2^-8 times the fp16 power of two 2^(ex - 119)
             const uint32_t f = (uint32_t)(ex - 104) << 10;
             const __half2 f2 = u2h(f | (f << 16));
 #pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-              o[2 * wi] = h2u(__hmul2(u2h(e4m3x2_bits_m8(__byte_perm(cw[wi], 0u, 0x4140))), f2));
-              o[2 * wi + 1] = h2u(__hmul2(u2h(e4m3x2_bits_m8(__byte_perm(cw[wi], 0u, 0x4342))), f2));
-            }
+            for (int k = 0; k < 4; ++k)
+              o[k] = h2u(__hmul2(u2h(e4m3x2_bits_m8(__byte_perm(w0, w1, k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12)))), f2));
           } else {
             // scales far from 1: fp32 product, rounded to fp16
             const float scf = exp2f((float)(ex - 127));
 #pragma unroll
-            for (int bb = 0; bb < 8; ++bb) {
-              const uint32_t two = (cw[bb >> 1] >> (16 * (bb & 1))) & 0xFFFF;
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t two = ((w0 >> (8 * k)) & 0xFF) | (((w1 >> (8 * k)) & 0xFF) << 8);
               const float2 f = __half22float2(dec_e4m3x2(two));
-              o[bb] = h2u(__floats2half2_rn(f.x * scf, f.y * scf));
+              o[k] = h2u(__floats2half2_rn(f.x * scf, f.y * scf));
             }
           }
-#pragma unroll
-          for (int half8 = 0; half8 < 2; ++half8) {
-            const int d = 128 * q4 + 16 * k + 8 * half8;
-            *reinterpret_cast<uint4*>(kt + (uint32_t)(d >> 6) * kAtKVBlk + sw128_offset_h(e, d & 63)) =
-                make_uint4(o[4 * half8], o[4 * half8 + 1], o[4 * half8 + 2], o[4 * half8 + 3]);
-          }
+          const int d = 128 * q4 + 8 * g;
+          *reinterpret_cast<uint4*>(kt + (uint32_t)(d >> 6) * kAtKVBlk + sw128_offset_h(e, d & 63)) =
+              make_uint4(o[0], o[1], o[2], o[3]);
         }
       } else {
 #pragma unroll
@@ -337,7 +380,6 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       if (lane == 0) mbar_arrive(kv_full + bi);
       if (i + 1 < nt) CSA_AT_FETCH(tile0 + i + 1);
     }
-#undef CSA_AT_FETCH
   } else {
     // ---------------------------------------------------------------- softmax
     const int qtr = warp;                      // TMEM lanes 32*qtr .. +31
@@ -347,41 +389,52 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     const float sc_main = p.scale_log2 * 128.f, sc_win = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;      // l_run: this lane's entry half
     bool ok = true;
-    // selected position of entry `lane` of the next tile (window entries: row exists)
-    int pos_next = 0;
-    if (nt > 0) {
-      const int jj = tile0 * kAtE + lane;
-      pos_next = jj < p.K ? idx_b[jj] : (jj < p.n_entries ? 0 : -1);
-    }
+    // selected positions of entries `lane` and `lane + 32` of the next tile
+    // (window entries: 0 when the row exists)
+    int pos_a = -1, pos_b = -1;
+    auto load_pos = [&](int tile) {
+      const int ja = tile * kAtE + lane, jb = ja + 32;
+      pos_a = ja < p.K ? idx_b[ja] : (ja < p.n_entries ? 0 : -1);
+      pos_b = jb < p.K ? idx_b[jb] : (jb < p.n_entries ? 0 : -1);
+    };
+    if (nt > 0) load_pos(tile0);
     for (int i = 0; i < nt; ++i) {
       const int bi = i & 1;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, pos_next >= 0);
-      if (i + 1 < nt) {
-        const int jj = (tile0 + i + 1) * kAtE + lane;
-        pos_next = jj < p.K ? idx_b[jj] : (jj < p.n_entries ? 0 : -1);
-      }
+      const uint32_t vm_a = __ballot_sync(0xffffffffu, pos_a >= 0);
+      const uint32_t vm_b = __ballot_sync(0xffffffffu, pos_b >= 0);
+      if (i + 1 < nt) load_pos(tile0 + i + 1);
       // a failed wait leaves `ok` false and skips the later waits, but every
       // warp still passes the group's named barriers once per tile
-      ok = ok && mbar_wait_warp(s_full + bi, (uint32_t)(i >> 1) & 1u, kErrWaitAccFull);
+      ok = ok && mbar_wait_warp(s_full, (uint32_t)i & 1u, kErrWaitAccFull);
       tc_fence_after();
-      float sv[kAtE];
-#pragma unroll
-      for (int k = 0; k < kAtE / 16; ++k) tmem_ld16f(trow + 32u * bi + 16 * k, sv + 16 * k);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free + bi);
-      // this lane takes entries [16*part, 16*part + 16): add the partner row's part
-      const int jbase = (tile0 + i) * kAtE + 16 * part;
+      // this lane takes entries [32*part, 32*part + 32) and adds the partner
+      // row's logits for them; 16 columns per round keeps the live registers low
+      const uint32_t vmask = part ? vm_b : vm_a;
+      const int jbase = (tile0 + i) * kAtE + 32 * part;
       const int n_main = p.K - jbase;          // entries below n_main are main (FP4) entries
-      float x[16];
+      float x[32];
+#pragma unroll
+      for (int rnd = 0; rnd < 4; ++rnd) {
+        float sv[16];
+        tmem_ld16f(trow + kAtSCol + 16 * rnd, sv);
+        tmem_wait_ld();
+        if (rnd == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+        }
+        const bool mine = (rnd >> 1) == part;   // columns 16rnd.. are this lane's entries
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float sum = sv[k] + __shfl_xor_sync(0xffffffffu, sv[k], 1);
+          const int en = 16 * (rnd & 1) + k;
+          if (mine) x[en] = sum;
+        }
+      }
       float mt = -INFINITY;
 #pragma unroll
-      for (int en = 0; en < 16; ++en) {
-        const float send = part ? sv[en] : sv[16 + en];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-        const float sum = (part ? sv[16 + en] : sv[en]) + recv;
-        const float v = ((vmask >> (16 * part + en)) & 1u) ? sum * (en < n_main ? sc_main : sc_win) : -INFINITY;
+      for (int en = 0; en < 32; ++en) {
+        const float v = ((vmask >> en) & 1u) ? x[en] * (en < n_main ? sc_main : sc_win) : -INFINITY;
         x[en] = v;
         mt = fmaxf(mt, v);
       }
@@ -393,10 +446,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
         m_run = mt;
         need = i > 0;
       }
-      if (part == 0) S.alpha_s[hp] = alpha;
+      // rescale factors by tile parity: after this tile's reduction barrier a
+      // warp may already write the next tile's factors while another still
+      // reads these
+      if (part == 0) S.alpha_s[64 * bi + hp] = alpha;
       float ls = 0.f;
 #pragma unroll
-      for (int en = 0; en < 16; ++en) {
+      for (int en = 0; en < 32; ++en) {
         const float pe = (m_run == -INFINITY) ? 0.f : ex2_approx(x[en] - m_run);
         ls += pe;
         x[en] = en < n_main ? pe * 128.f : pe;
@@ -405,13 +461,24 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       // the P buffer is free once the PV two tiles back has retired
       if (i >= 2) ok = ok && mbar_wait_warp(kv_free + bi, (uint32_t)((i >> 1) - 1) & 1u, kErrWaitSmemEmpty);
       {
-        uint8_t* pt = S.p + bi * kAtPBytes;
+        // P as fp16 hi + lo parts (~22 bits): with fp16 P alone the weights'
+        // rounding (2^-12) shows in channels whose entries are large but
+        // whose weighted sum cancels
+        uint8_t* pt = S.p + bi * 2 * kAtPBytes;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t o[4];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t oh[4], ol[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) o[k] = h2u(__floats2half2_rn(x[8 * c + 2 * k], x[8 * c + 2 * k + 1]));
-          *reinterpret_cast<uint4*>(pt + sw64_offset(hp, 32 * part + 16 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
+          for (int k = 0; k < 4; ++k) {
+            const float a0 = x[8 * c + 2 * k], a1 = x[8 * c + 2 * k + 1];
+            const __half2 hh = __floats2half2_rn(a0, a1);
+            const float2 hf = __half22float2(hh);
+            oh[k] = h2u(hh);
+            ol[k] = h2u(__floats2half2_rn(a0 - hf.x, a1 - hf.y));
+          }
+          const uint32_t off = sw128_offset_h(hp, 32 * part + 8 * c);
+          *reinterpret_cast<uint4*>(pt + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+          *reinterpret_cast<uint4*>(pt + kAtPBytes + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
         }
       }
       // any head whose running max moved rescales the accumulated O^T columns
@@ -422,16 +489,20 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       if (any_need) {
         ok = ok && mbar_wait_warp(o_done, (uint32_t)(i - 1) & 1u, kErrWaitAccFull);
         tc_fence_after();
+        // 16 heads at a time: their factors stay in registers across the 4 chunks
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int k = 0; k < 4; ++k) {
+          float al[16];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int cc = 0; cc < 16; ++cc) al[cc] = S.alpha_s[64 * bi + 16 * k + cc];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
             const uint32_t ta = trow + kAtOCol + 64 * c + 16 * k;
             uint32_t o[16];
             tmem_ld16(ta, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * S.alpha_s[16 * k + cc]);
+            for (int cc = 0; cc < 16; ++cc) o[cc] = __float_as_uint(__uint_as_float(o[cc]) * al[cc]);
             tmem_st16(ta, o);
           }
         }
@@ -444,10 +515,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     const int h = hp;
-    const bool is_hi = part == 0;
     // ------------------------------------------------------------- output
     // per-head output scale (normalised, sink folded in) and lse, or partials
-    if (is_hi) {
+    if (part == 0) {
       float scl = 1.f;
       if (p.n_splits == 1) {
         float m0 = m_run, l0 = l_run;
@@ -472,14 +542,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     if (ok && nt > 0) ok = mbar_wait_warp(o_done, ((uint32_t)(nt - 1) & 1u), kErrWaitAccFull);
     tc_fence_after();
     for (int c = 0; c < 4; ++c) {
-      const int d = 128 * c + 32 * qtr + lane;
+      // O^T row (position) 128c + 32qtr + lane holds this latent channel
+      const int dp = 128 * c + 32 * qtr + lane;
+      const int d = (dp & ~7) | perm8(dp & 7);
       // 64 heads of channel d: four loads in flight, one wait
       uint32_t o[64];
       if (nt > 0 && ok) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           uint32_t (&ok16)[16] = *reinterpret_cast<uint32_t(*)[16]>(o + 16 * k);
-          tmem_ld16(tbase + ((uint32_t)(32 * qtr) << 16) + kAtOCol + 64 * c + 16 * k, ok16);
+          tmem_ld16(trow + kAtOCol + 64 * c + 16 * k, ok16);
         }
         tmem_wait_ld();
       } else {
@@ -497,9 +569,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       }
     }
   }
+#undef CSA_AT_FETCH
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == kAtWarpS) {
     tc_fence_after();
     tmem_dealloc(tbase, kAtTmemCols);
   }

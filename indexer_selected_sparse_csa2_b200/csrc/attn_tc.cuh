@@ -21,7 +21,7 @@ struct AttnTcParams {
   float* out;
   float* lse;
   int n_entries;
-  int tiles_per_split;        // in 32-entry tiles
+  int tiles_per_split;        // in 64-entry tiles
   int n_splits;
   float* part_o;              // [B*n_q][n_splits][64][512] when n_splits > 1
   float* part_ml;             // [B*n_q][n_splits][64][2]

@@ -246,7 +246,7 @@ CSA_DEV void write_selected(const SelectJob& J, int b, uint32_t j, int32_t slot)
   }
 }
 
-__global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs jobs) {
+__global__ void __launch_bounds__(kFinalThreads, 1) select_final_kernel(SelectJobs jobs) {
   pdl_enter();
   const SelectJob& J = jobs.j[blockIdx.y];
   const int b = blockIdx.x;
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs 
   __shared__ uint32_t total;
   __shared__ uint32_t hist[256];
   __shared__ uint32_t s_prefix, s_krem;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int nruns = J.nchunks;
   const int32_t* cnt_row = J.cnt + (int64_t)b * nruns;
 
@@ -283,19 +283,39 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectJobs 
   }
   __syncthreads();
 
-  // 2. contiguous ordered list (shared memory when it fits); warp w copies
-  //    runs w, w + 32, ...
+  // 2. contiguous ordered list (shared memory when it fits).  List element i
+  //    comes from the last run r with offs[r] <= i (a binary search over the
+  //    run offsets; runs past nruns hold offset m); each thread moves four
+  //    elements per round so their loads are in flight together.
   const bool in_smem = m <= (uint32_t)kListCap;
   uint32_t* lk = in_smem ? skey : J.list_key + (int64_t)b * J.n;
   int32_t* lp = in_smem ? spos : J.list_pos + (int64_t)b * J.n;
-  for (int r = warp; r < nruns; r += kFinalThreads / 32) {
-    const uint32_t n_r = (uint32_t)cnt_row[r];
-    const uint32_t* src_k = J.cand_key + (int64_t)b * J.n + (int64_t)r * J.chunk;
-    const int32_t* src_p = J.cand_pos + (int64_t)b * J.n + (int64_t)r * J.chunk;
-    const uint32_t o = offs[r];
-    for (uint32_t i = lane; i < n_r; i += 32) {
-      lk[o + i] = src_k[i];
-      lp[o + i] = src_p[i];
+  {
+    const uint32_t* ck = J.cand_key + (int64_t)b * J.n;
+    const int32_t* cp = J.cand_pos + (int64_t)b * J.n;
+    for (uint32_t i0 = tid; i0 < m; i0 += 4 * kFinalThreads) {
+      int64_t src[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * kFinalThreads;
+        int r = 0;   // invariant offs[r] <= i; r + step <= kMaxRuns - 1 at every step
+#pragma unroll
+        for (int step = kMaxRuns / 2; step >= 1; step >>= 1)
+          if (offs[r + step] <= i) r += step;
+        src[u] = (int64_t)r * J.chunk + (i - offs[r]);
+      }
+      uint32_t kk[4];
+      int32_t pp[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * kFinalThreads;
+        if (i < m) { kk[u] = ck[src[u]]; pp[u] = cp[src[u]]; }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * kFinalThreads;
+        if (i < m) { lk[i] = kk[u]; lp[i] = pp[u]; }
+      }
     }
   }
   __syncthreads();
