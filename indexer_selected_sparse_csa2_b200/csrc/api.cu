@@ -12,6 +12,7 @@
 #include <atomic>
 
 #include "select.cuh"
+#include "quant.cuh"
 
 namespace csa {
 
@@ -21,7 +22,8 @@ void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_
 cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
                          int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream);
 size_t index_decode_ws_bytes(const csa_index_args* a);
-cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream);
+cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists);
+size_t index_hist_bytes(const csa_index_args* a);
 size_t attn_ws_bytes(const csa_attn_args* a);
 int read_tc_error(bool clear);
 int read_pf_error(bool clear);
@@ -128,7 +130,7 @@ csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t works
   const size_t need = index_decode_ws_bytes(a);
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
-  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream));
+  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream, nullptr));
 }
 
 size_t csa_topk_workspace_size(int32_t B, int64_t n) {
@@ -211,28 +213,16 @@ static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_ar
   return CSA_OK;
 }
 
-size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) {
-  if (!layers || n_layers < 1) return 0;
-  size_t need = 0;
-  for (int32_t i = 0; i < n_layers; ++i) {
-    csa_index_args ix{};
-    csa_attn_args at{};
-    if (resolve_layer(layers, i, &ix, &at) != CSA_OK) return 0;
-    if (layers[i].mode != CSA_MODE_REUSE) {
-      if (check_index(&ix) != CSA_OK) return 0;
-      need = std::max(need, index_decode_ws_bytes(&ix));
-    }
-    if (check_attn(&at) != CSA_OK) return 0;
-    need = std::max(need, attn_ws_bytes(&at));
-  }
-  return need;
-}
+// Workspace of a layer stack: the largest per-layer need (the layers run one
+// after another and share it), then one histogram region per indexed decode
+// layer, all cleared by the stack's single prologue launch.
+struct StackWs {
+  size_t main = 0;         // shared part
+  size_t hists = 0;        // total of the per-layer histogram regions
+};
 
-csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
-                          size_t workspace_bytes, csa_stream_t stream) {
-  if (!layers || n_layers < 1) return CSA_ERR_INVALID_ARG;
-  // validate everything before enqueuing anything
-  size_t need = 0;
+static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, StackWs* out) {
+  StackWs w;
   for (int32_t i = 0; i < n_layers; ++i) {
     csa_index_args ix{};
     csa_attn_args at{};
@@ -247,28 +237,79 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     if (layers[i].mode != CSA_MODE_REUSE) {
       s = check_index(&ix);
       if (s != CSA_OK) return s;
-      need = std::max(need, index_decode_ws_bytes(&ix));
+      w.main = std::max(w.main, index_decode_ws_bytes(&ix));
+      w.hists += index_hist_bytes(&ix);
     }
     s = check_attn(&at);
     if (s != CSA_OK) return s;
-    need = std::max(need, attn_ws_bytes(&at));
+    w.main = std::max(w.main, attn_ws_bytes(&at));
   }
+  w.main = (w.main + 255) & ~(size_t)255;
+  *out = w;
+  return CSA_OK;
+}
+
+size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) {
+  if (!layers || n_layers < 1) return 0;
+  StackWs w;
+  if (stack_ws(layers, n_layers, &w) != CSA_OK) return 0;
+  return w.main + w.hists;
+}
+
+csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
+                          size_t workspace_bytes, csa_stream_t stream) {
+  if (!layers || n_layers < 1) return CSA_ERR_INVALID_ARG;
+  // validate everything before enqueuing anything
+  StackWs w;
+  csa_status s = stack_ws(layers, n_layers, &w);
+  if (s != CSA_OK) return s;
+  const size_t need = w.main + w.hists;
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
+  uint8_t* hist_base = static_cast<uint8_t*>(workspace) + w.main;
+
+  // prologue: every layer's appended rows and the clearing of every layer's
+  // histograms, in one launch (each layer reads only rows appended before it
+  // in stream order, so moving the appends ahead of all layers is the same)
+  QuantBatch qb{};
+  qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
+  qb.zero_n16 = (int64_t)(w.hists / 16);
+  for (int32_t i = 0; i < n_layers; ++i) {
+    for (int k = 0; k < 3; ++k) {
+      const csa_quant_job& q = layers[i].append[k];
+      if (!q.src || q.n_rows == 0) continue;
+      if (qb.njobs == kMaxBatchJobs) {
+        if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
+        qb.njobs = 0;
+        qb.units = 0;
+        qb.zero_n16 = 0;
+      }
+      QuantBatchJob& J = qb.job[qb.njobs++];
+      const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
+      J.src = q.src;
+      J.n_rows = q.n_rows;
+      J.src_stride_bytes = q.src_row_stride * esz;
+      J.dst = static_cast<uint8_t*>(q.dst);
+      J.dst_stride = q.dst_row_stride;
+      J.fmt = q.fmt;
+      J.bf16 = q.src_dtype == CSA_SRC_BF16;
+      J.dim = q.dim;
+      J.unit0 = qb.units;
+      qb.units += quant_batch_units(q.fmt, q.n_rows, q.dim);
+    }
+  }
+  if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
+
+  size_t hist_off = 0;
   for (int32_t i = 0; i < n_layers; ++i) {
     csa_index_args ix{};
     csa_attn_args at{};
     resolve_layer(layers, i, &ix, &at);
-    for (int k = 0; k < 3; ++k) {
-      const csa_quant_job& q = layers[i].append[k];
-      if (!q.src || q.n_rows == 0) continue;
-      if (launch_quant(q.src, q.src_dtype, q.n_rows, q.dim, q.src_row_stride, q.fmt, q.dst, q.dst_row_stride,
-                       st) != cudaSuccess)
-        return CSA_ERR_CUDA;
-    }
     if (layers[i].mode != CSA_MODE_REUSE) {
-      if (run_index_decode(&ix, workspace, st) != cudaSuccess) return CSA_ERR_CUDA;
+      uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
+      hist_off += index_hist_bytes(&ix);
+      if (run_index_decode(&ix, workspace, st, h) != cudaSuccess) return CSA_ERR_CUDA;
     }
     if (run_sparse_attn(&at, workspace, st) != cudaSuccess) return CSA_ERR_CUDA;
   }

@@ -239,15 +239,27 @@ size_t index_decode_ws_bytes(const csa_index_args* a) {
   return carve_index_ws(a, nullptr).bytes;
 }
 
-cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream) {
+size_t index_hist_bytes(const csa_index_args* a) {
+  return a->n_q > 1 ? 0 : al256((size_t)2 * a->B * kHistBins * 4);
+}
+
+// `hists`: optional region of index_hist_bytes(a) that the caller has already
+// cleared (a layer stack clears all its layers' histograms in one launch);
+// without it the workspace's own histograms are cleared here.
+cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists) {
   if (a->n_q > 1) return run_index_prefill(a, ws, stream);
   IndexWs w = carve_index_ws(a, ws);
   const int B = a->B;
   const int64_t n = a->pool ? (int64_t)a->pool_cap : a->T;
   cudaError_t e;
-  // histograms start at zero (both sit at the start of the workspace)
-  e = launch_zero(w.pos.hist, (size_t)(a->pool_out ? 2 : 1) * B * kHistBins * 4, stream);
-  if (e != cudaSuccess) return e;
+  if (hists) {
+    w.pos.hist = hists;
+    if (a->pool_out) w.blk.hist = hists + (size_t)B * kHistBins;
+  } else {
+    // histograms start at zero (both sit at the start of the workspace)
+    e = launch_zero(w.pos.hist, (size_t)(a->pool_out ? 2 : 1) * B * kHistBins * 4, stream);
+    if (e != cudaSuccess) return e;
+  }
   ScoreParams p{};
   p.keys = a->keys;
   p.key_row_stride = a->key_row_stride;

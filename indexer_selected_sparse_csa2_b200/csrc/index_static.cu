@@ -26,9 +26,6 @@
 
 namespace csa {
 
-size_t index_decode_ws_bytes(const csa_index_args* a);
-cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream);
-
 constexpr size_t kNoallocScratchBytes = (size_t)16 << 20;
 constexpr int kMaxDevices = 64;
 

@@ -11,6 +11,7 @@
 // i.e. exactly one FP4 scale block, or half of one FP8 scale block.  Rows are
 // read with 128-bit loads and written with 64/128-bit stores.
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace csa {
 
@@ -41,6 +42,29 @@ CSA_DEV void load16(const void* row, int lane, float (&x)[16]) {
   }
 }
 
+// One warp encodes row `row` of the source into one FP4 entry.
+template <int SRC>
+CSA_DEV void encode_fp4_row(const void* row, int lane, uint8_t* out) {
+  float x[16];
+  load16<SRC>(row, lane, x);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  const uint32_t s_code = enc_e4m3x2(0.f, __fdiv_rn(amax, 6.0f)) & 0xFF;
+  const float s = dec_e4m3(s_code);
+  uint32_t packed[2] = {0u, 0u};
+  if (s != 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // even channel in the low nibble
+      uint32_t b = enc_e2m1x2(__fdiv_rn(x[2 * i + 1], s), __fdiv_rn(x[2 * i], s));
+      packed[i >> 2] |= b << (8 * (i & 3));
+    }
+  }
+  *reinterpret_cast<uint2*>(out + 8 * lane) = make_uint2(packed[0], packed[1]);
+  out[256 + lane] = (uint8_t)s_code;
+}
+
 template <int SRC>
 __global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__ src, int64_t n_rows,
                                                         int64_t src_stride_bytes,
@@ -48,27 +72,8 @@ __global__ void __launch_bounds__(256) quant_fp4_kernel(const void* __restrict__
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
-    float x[16];
-    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, x);
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    const uint32_t s_code = enc_e4m3x2(0.f, __fdiv_rn(amax, 6.0f)) & 0xFF;
-    const float s = dec_e4m3(s_code);
-    uint32_t packed[2] = {0u, 0u};
-    if (s != 0.f) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        // even channel in the low nibble
-        uint32_t b = enc_e2m1x2(__fdiv_rn(x[2 * i + 1], s), __fdiv_rn(x[2 * i], s));
-        packed[i >> 2] |= b << (8 * (i & 3));
-      }
-    }
-    uint8_t* out = dst + r * dst_stride;
-    *reinterpret_cast<uint2*>(out + 8 * lane) = make_uint2(packed[0], packed[1]);
-    out[256 + lane] = (uint8_t)s_code;
-  }
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps)
+    encode_fp4_row<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, dst + r * dst_stride);
 }
 
 // Smallest e with amax <= 448 * 2^e, clamped to [-127, 127]; amax == 0 -> -127.
@@ -88,6 +93,28 @@ CSA_DEV float pow2f(int k) {
   return k >= -126 ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(1u << 22);
 }
 
+// One warp encodes one row into one FP8 window entry.
+template <int SRC>
+CSA_DEV void encode_fp8w_row(const void* row, int lane, uint8_t* out) {
+  float x[16];
+  load16<SRC>(row, lane, x);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 32-channel block = lane pair
+  const int e = ue8m0_exponent(amax);
+  const float sc = pow2f(-e);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo = enc_e4m3x2(x[4 * i + 1] * sc, x[4 * i + 0] * sc);
+    uint32_t hi = enc_e4m3x2(x[4 * i + 3] * sc, x[4 * i + 2] * sc);
+    w[i] = lo | (hi << 16);
+  }
+  *reinterpret_cast<uint4*>(out + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+  if ((lane & 1) == 0) out[512 + (lane >> 1)] = (uint8_t)(e + 127);
+}
+
 template <int SRC>
 __global__ void __launch_bounds__(256) quant_fp8w_kernel(const void* __restrict__ src, int64_t n_rows,
                                                          int64_t src_stride_bytes,
@@ -95,26 +122,24 @@ __global__ void __launch_bounds__(256) quant_fp8w_kernel(const void* __restrict_
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps) {
-    float x[16];
-    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, x);
-    float amax = 0.f;
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n_rows; r += warps)
+    encode_fp8w_row<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, dst + r * dst_stride);
+}
+
+// Plain E4M3 cast of 16 consecutive values (column group c of a row).
+template <int SRC>
+CSA_DEV void encode_plain16(const void* row, int c, uint8_t* out_row) {
+  float x[16];
+  // reuse the 16-value loader with "lane" = column group
+  load16<SRC>(row, c, x);
+  uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));   // 32-channel block = lane pair
-    const int e = ue8m0_exponent(amax);
-    const float sc = pow2f(-e);
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t lo = enc_e4m3x2(x[4 * i + 1] * sc, x[4 * i + 0] * sc);
-      uint32_t hi = enc_e4m3x2(x[4 * i + 3] * sc, x[4 * i + 2] * sc);
-      w[i] = lo | (hi << 16);
-    }
-    uint8_t* out = dst + r * dst_stride;
-    *reinterpret_cast<uint4*>(out + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-    if ((lane & 1) == 0) out[512 + (lane >> 1)] = (uint8_t)(e + 127);
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo = enc_e4m3x2(x[4 * i + 1], x[4 * i + 0]);
+    uint32_t hi = enc_e4m3x2(x[4 * i + 3], x[4 * i + 2]);
+    w[i] = lo | (hi << 16);
   }
+  *reinterpret_cast<uint4*>(out_row + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // Plain E4M3 cast: each thread encodes 16 consecutive values of one row.
@@ -129,18 +154,65 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(const void* __restrict
        g += (int64_t)gridDim.x * blockDim.x) {
     const int64_t r = g / per_row;
     const int c = (int)(g - r * per_row);
-    float x[16];
-    // reuse the 16-value loader with "lane" = column group
-    load16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, c, x);
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t lo = enc_e4m3x2(x[4 * i + 1], x[4 * i + 0]);
-      uint32_t hi = enc_e4m3x2(x[4 * i + 3], x[4 * i + 2]);
-      w[i] = lo | (hi << 16);
-    }
-    *reinterpret_cast<uint4*>(dst + r * dst_stride + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+    encode_plain16<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, c, dst + r * dst_stride);
   }
+}
+
+// ------------------------------------------------------------ batched jobs --
+// All the appends of a layer stack (and the clearing of its histogram
+// region) in one launch: a flat list of warp-sized units.  FP4 / FP8 rows
+// are one unit per row; plain casts pack 32 groups of 16 values per unit;
+// the zero range is 512 bytes per unit.
+__global__ void __launch_bounds__(256) quant_batch_kernel(QuantBatch qb) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t zero_units = (qb.zero_n16 + 31) / 32;
+  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < qb.units + zero_units;
+       u += warps) {
+    if (u >= qb.units) {
+      const int64_t i = (u - qb.units) * 32 + lane;
+      if (i < qb.zero_n16) qb.zero_ptr[i] = make_uint4(0, 0, 0, 0);
+      continue;
+    }
+    int j = 0;
+    while (j + 1 < qb.njobs && u >= qb.job[j + 1].unit0) ++j;
+    const QuantBatchJob& J = qb.job[j];
+    const int64_t lu = u - J.unit0;
+    const uint8_t* src = static_cast<const uint8_t*>(J.src);
+    if (J.fmt == CSA_FMT_FP4_E2M1_E4M3X16) {
+      if (J.bf16) encode_fp4_row<1>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
+      else encode_fp4_row<0>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
+    } else if (J.fmt == CSA_FMT_FP8_E4M3_UE8M0X32) {
+      if (J.bf16) encode_fp8w_row<1>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
+      else encode_fp8w_row<0>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
+    } else {
+      const int per_row = J.dim >> 4;
+      const int64_t g = lu * 32 + lane;
+      if (g < J.n_rows * per_row) {
+        const int64_t r = g / per_row;
+        const int c = (int)(g - r * per_row);
+        if (J.bf16) encode_plain16<1>(src + r * J.src_stride_bytes, c, J.dst + r * J.dst_stride);
+        else encode_plain16<0>(src + r * J.src_stride_bytes, c, J.dst + r * J.dst_stride);
+      }
+    }
+  }
+}
+
+int64_t quant_batch_units(int fmt, int64_t n_rows, int dim) {
+  if (fmt == CSA_FMT_FP8_E4M3_PLAIN) return (n_rows * (dim >> 4) + 31) / 32;
+  return n_rows;
+}
+
+cudaError_t launch_quant_batch(const QuantBatch& qb, cudaStream_t stream) {
+  const int64_t units = qb.units + (qb.zero_n16 + 31) / 32;
+  if (units == 0) return cudaSuccess;
+  int64_t g = (units + 7) / 8;
+  if (g > (int64_t)kNumSMs * 8) g = (int64_t)kNumSMs * 8;
+  ProfScope ps(stream, "quant_batch");
+  launch_k(quant_batch_kernel, dim3((unsigned)g), dim3(256), 0, stream, qb);
+  note_launches(1);
+  return cudaGetLastError();
 }
 
 static int grid_for(int64_t work, int per_block) {
