@@ -13,6 +13,7 @@
 
 #include "select.cuh"
 #include "quant.cuh"
+#include "q2.cuh"
 
 namespace csa {
 
@@ -28,7 +29,8 @@ size_t attn_ws_bytes(const csa_attn_args* a);
 int read_tc_error(bool clear);
 int read_pf_error(bool clear);
 int read_at_error(bool clear);
-cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream);
+cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2);
+bool attn_tc_path(const csa_attn_args* a);
 
 static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 static bool al16i(int64_t v) { return (v & 15) == 0; }
@@ -174,7 +176,7 @@ csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t works
   const size_t need = attn_ws_bytes(a);
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
-  return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream));
+  return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream, nullptr));
 }
 
 // Resolve one layer of a stack into concrete index / attention arguments.
@@ -219,7 +221,15 @@ static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_ar
 struct StackWs {
   size_t main = 0;         // shared part
   size_t hists = 0;        // total of the per-layer histogram regions
+  size_t q2 = 0;           // total of the per-layer staged decode queries
 };
+
+// Decode layers on the tcgen05 attention kernel get their queries staged by
+// the prologue (one copy per token instead of a conversion per split CTA).
+static size_t layer_q2_bytes(const csa_attn_args& at) {
+  if (at.n_q != 1 || !attn_tc_path(&at)) return 0;
+  return ((size_t)at.B * kQ2TokenBytes + 255) & ~(size_t)255;
+}
 
 static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, StackWs* out) {
   StackWs w;
@@ -243,6 +253,7 @@ static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, Stack
     s = check_attn(&at);
     if (s != CSA_OK) return s;
     w.main = std::max(w.main, attn_ws_bytes(&at));
+    w.q2 += layer_q2_bytes(at);
   }
   w.main = (w.main + 255) & ~(size_t)255;
   *out = w;
@@ -253,7 +264,7 @@ size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) 
   if (!layers || n_layers < 1) return 0;
   StackWs w;
   if (stack_ws(layers, n_layers, &w) != CSA_OK) return 0;
-  return w.main + w.hists;
+  return w.main + w.hists + w.q2;
 }
 
 csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
@@ -263,11 +274,12 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
   StackWs w;
   csa_status s = stack_ws(layers, n_layers, &w);
   if (s != CSA_OK) return s;
-  const size_t need = w.main + w.hists;
+  const size_t need = w.main + w.hists + w.q2;
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
   uint8_t* hist_base = static_cast<uint8_t*>(workspace) + w.main;
+  uint8_t* q2_base = hist_base + w.hists;
 
   // prologue: every layer's appended rows and the clearing of every layer's
   // histograms, in one launch (each layer reads only rows appended before it
@@ -275,33 +287,50 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
   QuantBatch qb{};
   qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
   qb.zero_n16 = (int64_t)(w.hists / 16);
+  auto add_job = [&](const void* src, int64_t n_rows, int64_t src_stride_bytes, void* dst, int64_t dst_stride,
+                     int fmt, int bf16, int dim) -> bool {
+    if (qb.njobs == kMaxBatchJobs) {
+      if (launch_quant_batch(qb, st) != cudaSuccess) return false;
+      qb.njobs = 0;
+      qb.units = 0;
+      qb.zero_n16 = 0;
+    }
+    QuantBatchJob& J = qb.job[qb.njobs++];
+    J.src = src;
+    J.n_rows = n_rows;
+    J.src_stride_bytes = src_stride_bytes;
+    J.dst = static_cast<uint8_t*>(dst);
+    J.dst_stride = dst_stride;
+    J.fmt = fmt;
+    J.bf16 = bf16;
+    J.dim = dim;
+    J.unit0 = qb.units;
+    qb.units += quant_batch_units(fmt, n_rows, dim);
+    return true;
+  };
+  size_t q2_off = 0;
   for (int32_t i = 0; i < n_layers; ++i) {
     for (int k = 0; k < 3; ++k) {
       const csa_quant_job& q = layers[i].append[k];
       if (!q.src || q.n_rows == 0) continue;
-      if (qb.njobs == kMaxBatchJobs) {
-        if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
-        qb.njobs = 0;
-        qb.units = 0;
-        qb.zero_n16 = 0;
-      }
-      QuantBatchJob& J = qb.job[qb.njobs++];
       const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
-      J.src = q.src;
-      J.n_rows = q.n_rows;
-      J.src_stride_bytes = q.src_row_stride * esz;
-      J.dst = static_cast<uint8_t*>(q.dst);
-      J.dst_stride = q.dst_row_stride;
-      J.fmt = q.fmt;
-      J.bf16 = q.src_dtype == CSA_SRC_BF16;
-      J.dim = q.dim;
-      J.unit0 = qb.units;
-      qb.units += quant_batch_units(q.fmt, q.n_rows, q.dim);
+      if (!add_job(q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
+                   q.src_dtype == CSA_SRC_BF16, q.dim))
+        return CSA_ERR_CUDA;
+    }
+    csa_index_args ix{};
+    csa_attn_args at{};
+    resolve_layer(layers, i, &ix, &at);
+    if (layer_q2_bytes(at)) {
+      if (!add_job(at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
+        return CSA_ERR_CUDA;
+      q2_off += layer_q2_bytes(at);
     }
   }
   if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
 
   size_t hist_off = 0;
+  q2_off = 0;
   for (int32_t i = 0; i < n_layers; ++i) {
     csa_index_args ix{};
     csa_attn_args at{};
@@ -311,7 +340,9 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       hist_off += index_hist_bytes(&ix);
       if (run_index_decode(&ix, workspace, st, h) != cudaSuccess) return CSA_ERR_CUDA;
     }
-    if (run_sparse_attn(&at, workspace, st) != cudaSuccess) return CSA_ERR_CUDA;
+    const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
+    q2_off += layer_q2_bytes(at);
+    if (run_sparse_attn(&at, workspace, st, q2) != cudaSuccess) return CSA_ERR_CUDA;
   }
   return CSA_OK;
 }

@@ -372,12 +372,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
 
 // Merge the per-split partial results (log-sum-exp combine): one CTA per
 // (token, head), 128 threads x 4 channels.
-__global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
+// One CTA per (token, head): 4 groups of 128 threads each take a quarter of
+// the splits for all 512 channels (4 per thread), so a thread keeps all of
+// its partial-O loads in flight at once; the groups' sums meet in shared
+// memory.  Split weights 2^(m_s - M) come from the (max, sum) partials.
+constexpr int kCombThreads = 512;
+constexpr int kCombGroups = kCombThreads / 128;
+__global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p) {
   pdl_enter();
   const int bt = blockIdx.x, h = blockIdx.y, H = p.H;
   const int S = p.n_splits;
   __shared__ float wgt_s[64];
   __shared__ float inv_s, max_s;
+  __shared__ float4 part[kCombGroups - 1][128];
   const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
   if (threadIdx.x < 32) {
     float M = sk;
@@ -400,23 +407,45 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AttnParams p) {
   }
   __syncthreads();
   const float M = max_s;
-  const int d = 4 * threadIdx.x;
+  const int grp = threadIdx.x >> 7, t = threadIdx.x & 127;
+  const int d = 4 * t;
+  auto weight = [&](int s) -> float {
+    if (S <= 64) return wgt_s[s];
+    const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
+    return m == -INFINITY ? 0.f : exp2f(m - M);
+  };
+  const float* po = p.part_o + ((int64_t)bt * S * H + h) * kD + d;
+  const int64_t sstride = (int64_t)H * kD;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < S; ++s) {
-    float w;
-    if (S <= 64) {
-      w = wgt_s[s];
-    } else {
-      const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
-      w = m == -INFINITY ? 0.f : exp2f(m - M);
+  // this group's splits grp, grp + 4, ...: up to 10 loads in flight per round
+  constexpr int kR = 10;
+  for (int s0 = grp; s0 < S; s0 += kR * kCombGroups) {
+    uint4 v[kR];
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int s = s0 + k * kCombGroups;
+      v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
     }
-    if (w == 0.f) continue;
-    const float4 v = *reinterpret_cast<const float4*>(p.part_o + (((int64_t)bt * S + s) * H + h) * kD + d);
-    acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int s = s0 + k * kCombGroups;
+      const float w = s < S ? weight(s) : 0.f;
+      acc.x += w * __uint_as_float(v[k].x); acc.y += w * __uint_as_float(v[k].y);
+      acc.z += w * __uint_as_float(v[k].z); acc.w += w * __uint_as_float(v[k].w);
+    }
   }
-  const float inv = inv_s;
-  *reinterpret_cast<float4*>(p.out + ((int64_t)bt * H + h) * kD + d) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (grp > 0) part[grp - 1][t] = acc;
+  __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int g = 0; g < kCombGroups - 1; ++g) {
+      const float4 o = part[g][t];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+    }
+    const float inv = inv_s;
+    *reinterpret_cast<float4*>(p.out + ((int64_t)bt * H + h) * kD + d) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  }
 }
 
 template <int H>
@@ -430,14 +459,18 @@ struct AttnPlan {
   int tiles_per_split;
 };
 
+static bool use_tc_attention();
+
 static AttnPlan plan_attn(const csa_attn_args* a) {
   AttnPlan pl;
   const int n_entries = a->K + a->n_win;
   const int n_tiles = (n_entries + kTileE - 1) / kTileE;
   const int64_t tokens = (int64_t)a->B * a->n_q;
   int want = (int)((kNumSMs + tokens - 1) / tokens);
-  // at least two tiles per split: each split reloads q and writes a partial O
-  const int by_tiles = (n_tiles + 1) / 2;
+  // at least two tiles per split on the mma.sync kernel (each split reloads q
+  // and writes a partial O); the tcgen05 kernel takes single tiles, its
+  // per-split cost is small next to a tile's latency
+  const int by_tiles = (a->H == 64 && use_tc_attention()) ? n_tiles : (n_tiles + 1) / 2;
   if (want > by_tiles) want = by_tiles;
   if (want < 1) want = 1;
   if (want > n_tiles) want = n_tiles > 0 ? n_tiles : 1;
@@ -469,7 +502,7 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   note_launches(1);
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    launch_k(attn_combine_kernel, dim3(dim3(p.B * p.n_q, H)), dim3(128), 0, stream, p);
+    launch_k(attn_combine_kernel, dim3(dim3(p.B * p.n_q, H)), dim3(kCombThreads), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();
@@ -488,8 +521,9 @@ static bool use_tc_attention() {
 
 
 // 64 heads run on the tcgen05 kernel; other head counts on the mma.sync kernel.
-static cudaError_t launch_attn_64_tc(AttnParams& p, cudaStream_t stream) {
+static cudaError_t launch_attn_64_tc(AttnParams& p, const void* q2, cudaStream_t stream) {
   AttnTcParams t;
+  t.q2 = static_cast<const uint8_t*>(q2);
   t.B = p.B; t.n_q = p.n_q; t.q = p.q; t.kv = p.kv; t.kv_row_stride = p.kv_row_stride;
   t.kv_batch_stride = p.kv_batch_stride; t.idx = p.idx; t.K = p.K; t.win = p.win;
   t.win_row_stride = p.win_row_stride; t.win_batch_stride = p.win_batch_stride; t.n_win = p.n_win;
@@ -502,13 +536,17 @@ static cudaError_t launch_attn_64_tc(AttnParams& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, 64), dim3(128), 0, stream, p);
+    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, 64), dim3(kCombThreads), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();
 }
 
-cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream) {
+// True when these arguments run on the tcgen05 kernel (which can take q
+// already staged by a layer stack's prologue).
+bool attn_tc_path(const csa_attn_args* a) { return a->H == 64 && use_tc_attention(); }
+
+cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2) {
   AttnPlan pl = plan_attn(a);
   AttnParams p{};
   p.B = a->B; p.n_q = a->n_q; p.H = a->H;
@@ -531,7 +569,7 @@ cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t strea
   switch (a->H) {
     case 16: return launch_attn_h<16>(p, stream);
     case 32: return launch_attn_h<32>(p, stream);
-    case 64: return use_tc_attention() ? launch_attn_64_tc(p, stream) : launch_attn_h<64>(p, stream);
+    case 64: return use_tc_attention() ? launch_attn_64_tc(p, q2, stream) : launch_attn_h<64>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

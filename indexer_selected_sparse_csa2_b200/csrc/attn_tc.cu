@@ -38,6 +38,7 @@
 // probabilities by 2^7 in P, which leaves S and O unchanged.  Window entries
 // are staged unscaled.  All waits are bounded (sm100.cuh).
 #include "sm100.cuh"
+#include "q2.cuh"
 #include "attn_tc.cuh"
 
 namespace csa {
@@ -92,9 +93,6 @@ CSA_DEV AtSmem carve_at(uint8_t* raw) {
 CSA_DEV uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 CSA_DEV __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Channel held at position p (0..7) of an 8-channel group.
-CSA_DEV int perm8(int p) { return (p >> 1) + 4 * (p & 1); }
-
 // Integer-pipe decoders (the conversion pipe is the scarce one here).
 // An 8-bit E4M3 code c at bits 0-7 (and 16-23) becomes the fp16 value
 // E4M3(c) * 2^-8 by moving exponent and mantissa up by 7 and the sign to bit
@@ -119,22 +117,6 @@ CSA_DEV float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// fp16 hi / lo parts of 8 channels (a: channels 0-3, c: 4-7) in the staged
-// order, as four packed pairs.
-CSA_DEV void q_hilo_perm8(float4 a, float4 c, bool lo, uint32_t (&o)[4]) {
-  const float f0[4] = {a.x, a.y, a.z, a.w}, f1[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const __half2 hi = __floats2half2_rn(f0[k], f1[k]);       // channels k, k + 4
-    if (!lo) {
-      o[k] = h2u(hi);
-    } else {
-      const float2 hf = __half22float2(hi);
-      o[k] = h2u(__floats2half2_rn(f0[k] - hf.x, f1[k] - hf.y));
-    }
-  }
-}
-
 // Bounded wait taken by a whole warp; the result is the same in every lane, so
 // the warp-collective TMEM accesses after it stay convergent on every path.
 CSA_DEV bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int code) {
@@ -203,9 +185,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       kind = 2;                                                                                \
     }                                                                                          \
   } while (0)
-  // the first tile's entries are in flight while q is staged
   const bool is_deq = warp >= 4 && warp < kAtWarpS;
-  if (is_deq && nt > 0) CSA_AT_FETCH(tile0);
 
   if (warp == kAtWarpS) tmem_alloc(S.tmem_base, kAtTmemCols);
   tc_fence_before();
@@ -218,6 +198,41 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   // g = j / 4; lane quarter qq is written by warps qq, qq + 4 and qq + 8, four
   // 16-column stores each.
   const float* qg = p.q + (int64_t)bt * kAtH * kD;
+  if (p.q2) {
+    // q staged by the stack prologue: copy rows into TMEM, the rest into shared memory
+    const uint8_t* q2t = p.q2 + (size_t)bt * kQ2TokenBytes;
+    if (warp < kAtWarpS) {
+      const int qq = warp & 3, wr = warp >> 2;
+      const int r = 32 * qq + lane;
+      const uint4* src = reinterpret_cast<const uint4*>(q2t + ((size_t)r * kQ2TmemWords + 64 * wr) * 4);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {          // 8 loads in flight per half
+        uint4 f[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) f[k] = ld_nc_v4(src + 8 * half + k);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint32_t v[16];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            v[4 * k] = f[4 * u + k].x; v[4 * k + 1] = f[4 * u + k].y;
+            v[4 * k + 2] = f[4 * u + k].z; v[4 * k + 3] = f[4 * u + k].w;
+          }
+          tmem_st16(tbase + ((uint32_t)(32 * qq) << 16) + 64u * wr + 32u * half + 16u * u, v);
+        }
+      }
+      tmem_wait_st();
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(q2t + kQ2TmemBytes);
+    uint4* dst = reinterpret_cast<uint4*>(S.q2);
+    constexpr int kN = kQ2SmemBytes / 16;
+    constexpr int kIt = (kN + kAtThreads - 1) / kAtThreads;
+    uint4 f[kIt];
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) if (tid + t * kAtThreads < kN) f[t] = ld_nc_v4(src + tid + t * kAtThreads);
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) if (tid + t * kAtThreads < kN) dst[tid + t * kAtThreads] = f[t];
+  } else {
   if (warp < kAtWarpS) {
     const int qq = warp & 3, wr = warp >> 2;
     const int r = 32 * qq + lane, h = r >> 1;
@@ -240,14 +255,33 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }
     tmem_wait_st();
   }
-  // shared part (channels 384..511): two K-major 128-byte-swizzled blocks
-  for (int i = tid; i < 128 * 16; i += kAtThreads) {
-    const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
-    const int h = r >> 1;
-    const float4* src = reinterpret_cast<const float4*>(qg + (int64_t)h * kD + 384 + 64 * kb + 8 * c8);
-    uint32_t o[4];
-    q_hilo_perm8(src[0], src[1], r & 1, o);
-    *reinterpret_cast<uint4*>(S.q2 + kb * kAtQBlkBytes + sw128_offset_h(r, 8 * c8)) = make_uint4(o[0], o[1], o[2], o[3]);
+  // shared part (channels 384..511): two K-major 128-byte-swizzled blocks;
+  // every load of a thread is issued before the first conversion
+  {
+    constexpr int kIt = (128 * 16 + kAtThreads - 1) / kAtThreads;
+    float4 f[2 * kIt];
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) {
+      const int i = tid + t * kAtThreads;
+      if (i < 128 * 16) {
+        const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
+        const float4* src = reinterpret_cast<const float4*>(qg + (int64_t)(r >> 1) * kD + 384 + 64 * kb + 8 * c8);
+        f[2 * t] = src[0];
+        f[2 * t + 1] = src[1];
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) {
+      const int i = tid + t * kAtThreads;
+      if (i < 128 * 16) {
+        const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
+        uint32_t o[4];
+        q_hilo_perm8(f[2 * t], f[2 * t + 1], r & 1, o);
+        *reinterpret_cast<uint4*>(S.q2 + kb * kAtQBlkBytes + sw128_offset_h(r, 8 * c8)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -313,6 +347,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }
   } else if (is_deq) {
     // --------------------------------------------------- gather + dequantise
+    if (nt > 0) CSA_AT_FETCH(tile0);
     for (int i = 0; i < nt; ++i) {
       const int bi = i & 1;
       if (i >= 2 && !mbar_wait_warp(kv_free + bi, (uint32_t)((i >> 1) - 1) & 1u, kErrWaitSmemEmpty)) break;

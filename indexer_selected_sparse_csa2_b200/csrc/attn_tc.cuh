@@ -23,6 +23,7 @@ struct AttnTcParams {
   int n_entries;
   int tiles_per_split;        // in 64-entry tiles
   int n_splits;
+  const uint8_t* q2;          // optional: q already staged (q2.cuh layout), [B*n_q] tokens
   float* part_o;              // [B*n_q][n_splits][64][512] when n_splits > 1
   float* part_ml;             // [B*n_q][n_splits][64][2]
 };

@@ -317,6 +317,8 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     jb.limit = a->T;
     jobs[nj++] = jb;
   }
+  // the Reindex layers' pool rows fit one CTA each
+  if (nj == 1 && select_small_ok(jobs[0])) return launch_select_small(jobs[0], B, stream);
   return launch_select(jobs, nj, B, false, stream);
 }
 

@@ -12,6 +12,7 @@
 // read with 128-bit loads and written with 64/128-bit stores.
 #include "common.cuh"
 #include "quant.cuh"
+#include "q2.cuh"
 
 namespace csa {
 
@@ -186,6 +187,10 @@ __global__ void __launch_bounds__(256) quant_batch_kernel(QuantBatch qb) {
     } else if (J.fmt == CSA_FMT_FP8_E4M3_UE8M0X32) {
       if (J.bf16) encode_fp8w_row<1>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
       else encode_fp8w_row<0>(src + lu * J.src_stride_bytes, lane, J.dst + lu * J.dst_stride);
+    } else if (J.fmt == kFmtStageQ2) {
+      const int64_t tok = lu >> 6;
+      encode_q2_head(reinterpret_cast<const float*>(src) + tok * (64 * 512), (int)(lu & 63), lane,
+                     J.dst + tok * kQ2TokenBytes);
     } else {
       const int per_row = J.dim >> 4;
       const int64_t g = lu * 32 + lane;

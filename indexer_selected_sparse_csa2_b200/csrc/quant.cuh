@@ -6,6 +6,10 @@
 namespace csa {
 
 constexpr int kMaxBatchJobs = 24;
+// Batch job format (besides the csa_kv_format values): stage a token's 64-head
+// attention query for the tcgen05 attention kernel (q2.cuh); n_rows = tokens
+// x 64 heads, src = fp32 queries [tokens][64][512], dst = [tokens][128 KB].
+constexpr int kFmtStageQ2 = 1000;
 
 struct QuantBatchJob {
   const void* src;
