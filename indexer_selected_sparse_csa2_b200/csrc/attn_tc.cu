@@ -443,27 +443,27 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       ok = ok && mbar_wait_warp(s_full, (uint32_t)i & 1u, kErrWaitAccFull);
       tc_fence_after();
       // this lane takes entries [32*part, 32*part + 32) and adds the partner
-      // row's logits for them; 16 columns per round keeps the live registers low
+      // row's logits for them; one 32-column load per half
       const uint32_t vmask = part ? vm_b : vm_a;
       const int jbase = (tile0 + i) * kAtE + 32 * part;
       const int n_main = p.K - jbase;          // entries below n_main are main (FP4) entries
       float x[32];
 #pragma unroll
-      for (int rnd = 0; rnd < 4; ++rnd) {
-        float sv[16];
-        tmem_ld16f(trow + kAtSCol + 16 * rnd, sv);
+      for (int rnd = 0; rnd < 2; ++rnd) {
+        uint32_t sv[32];
+        tmem_ld32(trow + kAtSCol + 32 * rnd, sv);
         tmem_wait_ld();
-        if (rnd == 3) {
+        if (rnd == 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
         }
-        const bool mine = (rnd >> 1) == part;   // columns 16rnd.. are this lane's entries
+        const bool mine = rnd == part;          // columns 32rnd.. are this lane's entries
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float sum = sv[k] + __shfl_xor_sync(0xffffffffu, sv[k], 1);
-          const int en = 16 * (rnd & 1) + k;
-          if (mine) x[en] = sum;
+        for (int k = 0; k < 32; ++k) {
+          const float v = __uint_as_float(sv[k]);
+          const float sum = v + __shfl_xor_sync(0xffffffffu, v, 1);
+          if (mine) x[k] = sum;
         }
       }
       float mt = -INFINITY;
@@ -580,14 +580,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       // O^T row (position) 128c + 32qtr + lane holds this latent channel
       const int dp = 128 * c + 32 * qtr + lane;
       const int d = (dp & ~7) | perm8(dp & 7);
-      // 64 heads of channel d: four loads in flight, one wait
+      // 64 heads of channel d: one 64-column load
       uint32_t o[64];
       if (nt > 0 && ok) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t (&ok16)[16] = *reinterpret_cast<uint32_t(*)[16]>(o + 16 * k);
-          tmem_ld16(trow + kAtOCol + 64 * c + 16 * k, ok16);
-        }
+        tmem_ld64(trow + kAtOCol + 64 * c, o);
         tmem_wait_ld();
       } else {
 #pragma unroll

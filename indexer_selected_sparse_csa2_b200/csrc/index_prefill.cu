@@ -230,32 +230,36 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
         if (!mbar_wait(&S.accf[a], (g / kPfAcc) & 1u, &g_pf_error, kErrWaitAccFull)) { failed = true; break; }
         tc_fence_after();
         const uint32_t col0 = tbase + ((uint32_t)(32 * quarter) << 16) + (uint32_t)(a * kPfN + qg * 64);
-        uint32_t r[4][16];
-        tmem_ld16(col0, r[0]);
-        tmem_ld16(col0 + 16, r[1]);
-        tmem_ld16(col0 + 32, r[2]);
-        tmem_ld16(col0 + 48, r[3]);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.acce[a]);
-        const int tile = MODE == 1 ? (int)x.kt0 + i : (int)pf_tile(p, x, i);
-        const int pos = tile * kPfRows + 32 * quarter + lane;
+        // two halves of 4 queries: one 32-column load each
         float sc[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 wa = wq[2 * k], wb = wq[2 * k + 1];
-          const uint32_t* rr = r[k >> 1] + (k & 1) * 8;
-          float2 acc = __fmul2_rn(make_float2(wa.x, wa.y), make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
-                                                                      fmaxf(__uint_as_float(rr[1]), 0.f)));
-          acc = __ffma2_rn(make_float2(wa.z, wa.w),
-                           make_float2(fmaxf(__uint_as_float(rr[2]), 0.f), fmaxf(__uint_as_float(rr[3]), 0.f)), acc);
-          acc = __ffma2_rn(make_float2(wb.x, wb.y),
-                           make_float2(fmaxf(__uint_as_float(rr[4]), 0.f), fmaxf(__uint_as_float(rr[5]), 0.f)), acc);
-          acc = __ffma2_rn(make_float2(wb.z, wb.w),
-                           make_float2(fmaxf(__uint_as_float(rr[6]), 0.f), fmaxf(__uint_as_float(rr[7]), 0.f)), acc);
-          sc[k] = acc.x + acc.y;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r32[32];
+          tmem_ld32(col0 + 32 * hf, r32);
+          tmem_wait_ld();
+          if (hf == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.acce[a]);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = 4 * hf + kk;
+            const float4 wa = wq[2 * k], wb = wq[2 * k + 1];
+            const uint32_t* rr = r32 + 8 * kk;
+            float2 acc = __fmul2_rn(make_float2(wa.x, wa.y), make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
+                                                                        fmaxf(__uint_as_float(rr[1]), 0.f)));
+            acc = __ffma2_rn(make_float2(wa.z, wa.w),
+                             make_float2(fmaxf(__uint_as_float(rr[2]), 0.f), fmaxf(__uint_as_float(rr[3]), 0.f)), acc);
+            acc = __ffma2_rn(make_float2(wb.x, wb.y),
+                             make_float2(fmaxf(__uint_as_float(rr[4]), 0.f), fmaxf(__uint_as_float(rr[5]), 0.f)), acc);
+            acc = __ffma2_rn(make_float2(wb.z, wb.w),
+                             make_float2(fmaxf(__uint_as_float(rr[6]), 0.f), fmaxf(__uint_as_float(rr[7]), 0.f)), acc);
+            sc[k] = acc.x + acc.y;
+          }
         }
+        const int tile = MODE == 1 ? (int)x.kt0 + i : (int)pf_tile(p, x, i);
+        const int pos = tile * kPfRows + 32 * quarter + lane;
         // visibility: every position of the tile is visible to every query
         // of the group unless the tile crosses the causal diagonal
         const bool all_vis = tile * kPfRows + kPfRows - 1 <= lim0;
