@@ -10,6 +10,7 @@
 // its own 128-token window).
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "select.cuh"
 #include "quant.cuh"
@@ -218,17 +219,29 @@ static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_ar
 // Workspace of a layer stack: the largest per-layer need (the layers run one
 // after another and share it), then one histogram region per indexed decode
 // layer, all cleared by the stack's single prologue launch.
+// Workspace of a layer stack: one region per layer (a layer's index scratch
+// and its attention partials; layers may run concurrently, so regions are not
+// shared), then one histogram region per indexed decode layer (all cleared by
+// the prologue launch), then the staged decode queries.
 struct StackWs {
-  size_t main = 0;         // shared part
+  size_t layers = 0;       // total of the per-layer regions
   size_t hists = 0;        // total of the per-layer histogram regions
   size_t q2 = 0;           // total of the per-layer staged decode queries
 };
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Decode layers on the tcgen05 attention kernel get their queries staged by
 // the prologue (one copy per token instead of a conversion per split CTA).
 static size_t layer_q2_bytes(const csa_attn_args& at) {
   if (at.n_q != 1 || !attn_tc_path(&at)) return 0;
-  return ((size_t)at.B * kQ2TokenBytes + 255) & ~(size_t)255;
+  return al256((size_t)at.B * kQ2TokenBytes);
+}
+
+static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& ix, const csa_attn_args& at) {
+  size_t r = attn_ws_bytes(&at);
+  if (L.mode != CSA_MODE_REUSE) r = std::max(r, index_decode_ws_bytes(&ix));
+  return al256(r);
 }
 
 static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, StackWs* out) {
@@ -247,15 +260,13 @@ static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, Stack
     if (layers[i].mode != CSA_MODE_REUSE) {
       s = check_index(&ix);
       if (s != CSA_OK) return s;
-      w.main = std::max(w.main, index_decode_ws_bytes(&ix));
       w.hists += index_hist_bytes(&ix);
     }
     s = check_attn(&at);
     if (s != CSA_OK) return s;
-    w.main = std::max(w.main, attn_ws_bytes(&at));
+    w.layers += layer_region_bytes(layers[i], ix, at);
     w.q2 += layer_q2_bytes(at);
   }
-  w.main = (w.main + 255) & ~(size_t)255;
   *out = w;
   return CSA_OK;
 }
@@ -264,26 +275,72 @@ size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) 
   if (!layers || n_layers < 1) return 0;
   StackWs w;
   if (stack_ws(layers, n_layers, &w) != CSA_OK) return 0;
-  return w.main + w.hists + w.q2;
+  return w.layers + w.hists + w.q2;
+}
+
+// Host-side streams and events the stack uses to run independent layers
+// concurrently (created once per device; no device memory).  Under stream
+// capture the fork / join below becomes graph edges.
+constexpr int kAuxStreams = 8;
+constexpr int kMaxStackLayers = 64;
+struct StackStreams {
+  cudaStream_t aux[kAuxStreams] = {};
+  cudaEvent_t pro = nullptr;
+  cudaEvent_t idx[kMaxStackLayers] = {};
+  cudaEvent_t done[kMaxStackLayers] = {};
+  bool ok = false;
+};
+static std::mutex g_stack_mu;
+static StackStreams g_stack[64];
+
+static StackStreams* stack_streams() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_stack_mu);
+  StackStreams& S = g_stack[dev];
+  if (!S.ok) {
+    bool good = true;
+    for (int i = 0; i < kAuxStreams && good; ++i)
+      good = cudaStreamCreateWithFlags(&S.aux[i], cudaStreamNonBlocking) == cudaSuccess;
+    good = good && cudaEventCreateWithFlags(&S.pro, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kMaxStackLayers && good; ++i)
+      good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&S.done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!good) return nullptr;
+    S.ok = true;
+  }
+  return &S;
+}
+
+// Source layer of a Reuse chain.
+static int32_t reuse_source(const csa_layer_desc* L, int32_t i) {
+  int32_t src = L[i].reuse_from;
+  while (L[src].mode == CSA_MODE_REUSE) src = L[src].reuse_from;
+  return src;
 }
 
 csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
                           size_t workspace_bytes, csa_stream_t stream) {
   if (!layers || n_layers < 1) return CSA_ERR_INVALID_ARG;
+  if (n_layers > kMaxStackLayers) return CSA_ERR_UNSUPPORTED;
   // validate everything before enqueuing anything
   StackWs w;
   csa_status s = stack_ws(layers, n_layers, &w);
   if (s != CSA_OK) return s;
-  const size_t need = w.main + w.hists + w.q2;
+  const size_t need = w.layers + w.hists + w.q2;
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
+  StackStreams* SS = stack_streams();
+  if (!SS) return CSA_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  uint8_t* hist_base = static_cast<uint8_t*>(workspace) + w.main;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* hist_base = base + w.layers;
   uint8_t* q2_base = hist_base + w.hists;
 
-  // prologue: every layer's appended rows and the clearing of every layer's
-  // histograms, in one launch (each layer reads only rows appended before it
-  // in stream order, so moving the appends ahead of all layers is the same)
+  // prologue: every layer's appended rows, the clearing of every layer's
+  // histograms and the staging of decode queries, in one launch (each layer
+  // reads only rows appended before it in stream order, so moving the appends
+  // ahead of all layers is the same)
   QuantBatch qb{};
   qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
   qb.zero_n16 = (int64_t)(w.hists / 16);
@@ -328,22 +385,40 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     }
   }
   if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
+  if (cudaEventRecord(SS->pro, st) != cudaSuccess) return CSA_ERR_CUDA;
 
-  size_t hist_off = 0;
+  // Layers run concurrently where the mode stack allows it: layer 0 on the
+  // caller's stream, layer i > 0 on an auxiliary stream that waits for the
+  // prologue, for the pool builder's Top-K (Reindex in a pool) or for the
+  // reused layer's Top-K (Reuse); the caller's stream then waits for all.
+  size_t reg_off = 0, hist_off = 0;
   q2_off = 0;
   for (int32_t i = 0; i < n_layers; ++i) {
     csa_index_args ix{};
     csa_attn_args at{};
     resolve_layer(layers, i, &ix, &at);
-    if (layers[i].mode != CSA_MODE_REUSE) {
+    const csa_layer_desc& L = layers[i];
+    cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kAuxStreams];
+    if (i > 0 && cudaStreamWaitEvent(ls, SS->pro, 0) != cudaSuccess) return CSA_ERR_CUDA;
+    uint8_t* region = base + reg_off;
+    reg_off += layer_region_bytes(L, ix, at);
+    if (L.mode != CSA_MODE_REUSE) {
+      if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->idx[L.pool_from], 0) != cudaSuccess)
+        return CSA_ERR_CUDA;
       uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
       hist_off += index_hist_bytes(&ix);
-      if (run_index_decode(&ix, workspace, st, h) != cudaSuccess) return CSA_ERR_CUDA;
+      if (run_index_decode(&ix, region, ls, h) != cudaSuccess) return CSA_ERR_CUDA;
+    } else if (cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
+      return CSA_ERR_CUDA;
     }
+    if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
     const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
     q2_off += layer_q2_bytes(at);
-    if (run_sparse_attn(&at, workspace, st, q2) != cudaSuccess) return CSA_ERR_CUDA;
+    if (run_sparse_attn(&at, region, ls, q2) != cudaSuccess) return CSA_ERR_CUDA;
+    if (i > 0 && cudaEventRecord(SS->done[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
   }
+  for (int32_t i = 1; i < n_layers; ++i)
+    if (cudaStreamWaitEvent(st, SS->done[i], 0) != cudaSuccess) return CSA_ERR_CUDA;
   return CSA_OK;
 }
 
