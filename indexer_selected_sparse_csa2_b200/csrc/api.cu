@@ -216,9 +216,6 @@ static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_ar
   return CSA_OK;
 }
 
-// Workspace of a layer stack: the largest per-layer need (the layers run one
-// after another and share it), then one histogram region per indexed decode
-// layer, all cleared by the stack's single prologue launch.
 // Workspace of a layer stack: one region per layer (a layer's index scratch
 // and its attention partials; layers may run concurrently, so regions are not
 // shared), then one histogram region per indexed decode layer (all cleared by

@@ -573,7 +573,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       S.scl[h] = scl;
     }
     named_bar(1, 128);
-    // every thread waits for the last PV itself (no wait is skipped on an error)
+    // every thread waits for the last PV itself (no wait is skipped on an error).
+    // o_done completes once per tile and a parity wait only tells the phase
+    // after the last completed one apart: the PV two tiles back is known
+    // retired (through kv_free), the one before the last is not (a last tile
+    // without a rescale never waited for it), so wait for both in order.
+    if (ok && nt > 1) ok = mbar_wait_warp(o_done, ((uint32_t)(nt - 2) & 1u), kErrWaitAccFull);
     if (ok && nt > 0) ok = mbar_wait_warp(o_done, ((uint32_t)(nt - 1) & 1u), kErrWaitAccFull);
     tc_fence_after();
     for (int c = 0; c < 4; ++c) {
