@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   uint64_t* s_free = S.bars + 5;     // S2 read by the softmax (4 warp arrivals)
   uint64_t* p_full = S.bars + 6;     // [2] P written, O^T rescaled (4 warp arrivals)
   uint64_t* o_done = S.bars + 8;     // one phase per PV
-  uint64_t* drain = S.bars + 9;      // [2] all MMAs of an issuer retired (teardown)
+  uint64_t* drain = S.bars + 9;      // [2] all MMAs of an issuer retired (teardown; [1] = every PV, for the output)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bt = blockIdx.y;
   const int b = bt / p.n_q, tq = bt - b * p.n_q;
@@ -573,13 +573,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       S.scl[h] = scl;
     }
     named_bar(1, 128);
-    // every thread waits for the last PV itself (no wait is skipped on an error).
-    // o_done completes once per tile and a parity wait only tells the phase
-    // after the last completed one apart: the PV two tiles back is known
-    // retired (through kv_free), the one before the last is not (a last tile
-    // without a rescale never waited for it), so wait for both in order.
-    if (ok && nt > 1) ok = mbar_wait_warp(o_done, ((uint32_t)(nt - 2) & 1u), kErrWaitAccFull);
-    if (ok && nt > 0) ok = mbar_wait_warp(o_done, ((uint32_t)(nt - 1) & 1u), kErrWaitAccFull);
+    // every thread waits for the last PV itself (no wait is skipped on an
+    // error), on the PV issuer's single-phase drain barrier: o_done completes
+    // once per tile and a parity wait on it cannot tell whether the PV before
+    // the last one has retired (a last tile without a rescale never waited
+    // for it), so it could return while that PV still accumulates.
+    if (ok && nt > 0) ok = mbar_wait_warp(drain + 1, 0u, kErrWaitAccFull);
     tc_fence_after();
     for (int c = 0; c < 4; ++c) {
       // O^T row (position) 128c + 32qtr + lane holds this latent channel

@@ -26,11 +26,17 @@ def csa():
     return m
 
 
-def _check_stack(csa, cfg, append=False, sinks=False, batches=None):
+def _check_stack(csa, cfg, append=False, sinks=False, batches=None, ws_fill=None):
     from csa_synth.device import DeviceCase
     dc = DeviceCase(cfg, sinks=sinks)
     descs = dc.layer_descs(append_rows=append)
-    csa.csa_layer_step(descs)
+    ws = None
+    if ws_fill is not None:
+        # a workspace whose every byte is set beforehand (the step must not
+        # depend on what it holds)
+        ws = torch.full((csa.csa_layer_workspace_size(descs),), ws_fill, dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+    csa.csa_layer_step(descs, workspace=ws)
     torch.cuda.synchronize()
     batches = range(cfg.B) if batches is None else batches
     for b in batches:
@@ -97,3 +103,25 @@ def test_hierarchical_small(csa):
 
 def test_hierarchical_ragged_tail(csa):
     _check_stack(csa, get_config("hier_1m", B=1, T=20003, pool_blocks=700, K=300))
+
+
+def test_cold_first_step(csa):
+    """The first step of a fresh process, on a workspace cleared just before
+    it: 8 decode tokens with 2 attention tiles per split, where the attention
+    epilogue must wait for the PV of the next-to-last tile as well as the last
+    (a cold step is where that PV still runs when the softmax warps finish)."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, CSA_COLD_STEP="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k", "cold_step_body"],
+                       env=env, capture_output=True, text=True, cwd=os.path.dirname(os.path.dirname(__file__)))
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+def test_cold_step_body(csa):
+    import os
+    if os.environ.get("CSA_COLD_STEP") != "1":
+        pytest.skip("runs in a fresh process under test_cold_first_step")
+    for fill in (0, 255):
+        _check_stack(csa, get_config("decode_64k", B=8, T=20000), append=True, ws_fill=fill)
