@@ -26,11 +26,11 @@ cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim
 size_t index_decode_ws_bytes(const csa_index_args* a);
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists);
 size_t index_hist_bytes(const csa_index_args* a);
-size_t attn_ws_bytes(const csa_attn_args* a);
+size_t attn_ws_bytes(const csa_attn_args* a, int share);
 int read_tc_error(bool clear);
 int read_pf_error(bool clear);
 int read_at_error(bool clear);
-cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2);
+cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2, int share);
 bool attn_tc_path(const csa_attn_args* a);
 
 static bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
@@ -167,17 +167,17 @@ csa_status csa_topk_scores(const float* scores, int32_t B, int64_t n, int64_t ro
 
 size_t csa_attn_workspace_size(const csa_attn_args* a) {
   if (check_attn(a) != CSA_OK) return 0;
-  return attn_ws_bytes(a);
+  return attn_ws_bytes(a, 1);
 }
 
 csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t workspace_bytes,
                            csa_stream_t stream) {
   csa_status s = check_attn(a);
   if (s != CSA_OK) return s;
-  const size_t need = attn_ws_bytes(a);
+  const size_t need = attn_ws_bytes(a, 1);
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (need && !al16(workspace)) return CSA_ERR_ALIGNMENT;
-  return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream, nullptr));
+  return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream, nullptr, 1));
 }
 
 // Resolve one layer of a stack into concrete index / attention arguments.
@@ -235,8 +235,34 @@ static size_t layer_q2_bytes(const csa_attn_args& at) {
   return al256((size_t)at.B * kQ2TokenBytes);
 }
 
-static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& ix, const csa_attn_args& at) {
-  size_t r = attn_ws_bytes(&at);
+// Source layer of a Reuse chain.
+static int32_t reuse_source(const csa_layer_desc* L, int32_t i) {
+  int32_t src = L[i].reuse_from;
+  while (L[src].mode == CSA_MODE_REUSE) src = L[src].reuse_from;
+  return src;
+}
+
+// Dependency wave of a layer of a validated stack: 0 for layers that wait only
+// for the prologue (Full, Reindex over all positions), otherwise one more than
+// the wave of the layer whose pool (Reindex in a pool) or Top-K (Reuse) it
+// waits for.  Layers of one wave run their attention at about the same time,
+// so each plans its split grid for its share of the SMs.
+static int layer_wave(const csa_layer_desc* L, int32_t i) {
+  if (L[i].mode == CSA_MODE_REUSE) return 1 + layer_wave(L, reuse_source(L, i));
+  if (L[i].mode == CSA_MODE_REINDEX && L[i].pool_from >= 0) return 1 + layer_wave(L, L[i].pool_from);
+  return 0;
+}
+
+static int attn_share(const csa_layer_desc* L, int32_t n_layers, int32_t i) {
+  const int w = layer_wave(L, i);
+  int c = 0;
+  for (int32_t j = 0; j < n_layers; ++j) c += layer_wave(L, j) == w;
+  return c;
+}
+
+static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& ix, const csa_attn_args& at,
+                                 int share) {
+  size_t r = attn_ws_bytes(&at, share);
   if (L.mode != CSA_MODE_REUSE) r = std::max(r, index_decode_ws_bytes(&ix));
   return al256(r);
 }
@@ -261,8 +287,14 @@ static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, Stack
     }
     s = check_attn(&at);
     if (s != CSA_OK) return s;
-    w.layers += layer_region_bytes(layers[i], ix, at);
     w.q2 += layer_q2_bytes(at);
+  }
+  // every layer is valid: the waves (and the split grids they set) are defined
+  for (int32_t i = 0; i < n_layers; ++i) {
+    csa_index_args ix{};
+    csa_attn_args at{};
+    resolve_layer(layers, i, &ix, &at);
+    w.layers += layer_region_bytes(layers[i], ix, at, attn_share(layers, n_layers, i));
   }
   *out = w;
   return CSA_OK;
@@ -307,13 +339,6 @@ static StackStreams* stack_streams() {
     S.ok = true;
   }
   return &S;
-}
-
-// Source layer of a Reuse chain.
-static int32_t reuse_source(const csa_layer_desc* L, int32_t i) {
-  int32_t src = L[i].reuse_from;
-  while (L[src].mode == CSA_MODE_REUSE) src = L[src].reuse_from;
-  return src;
 }
 
 csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
@@ -398,7 +423,8 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kAuxStreams];
     if (i > 0 && cudaStreamWaitEvent(ls, SS->pro, 0) != cudaSuccess) return CSA_ERR_CUDA;
     uint8_t* region = base + reg_off;
-    reg_off += layer_region_bytes(L, ix, at);
+    const int share = attn_share(layers, n_layers, i);
+    reg_off += layer_region_bytes(L, ix, at, share);
     if (L.mode != CSA_MODE_REUSE) {
       if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->idx[L.pool_from], 0) != cudaSuccess)
         return CSA_ERR_CUDA;
@@ -411,7 +437,7 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
     const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
     q2_off += layer_q2_bytes(at);
-    if (run_sparse_attn(&at, region, ls, q2) != cudaSuccess) return CSA_ERR_CUDA;
+    if (run_sparse_attn(&at, region, ls, q2, share) != cudaSuccess) return CSA_ERR_CUDA;
     if (i > 0 && cudaEventRecord(SS->done[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
   }
   for (int32_t i = 1; i < n_layers; ++i)

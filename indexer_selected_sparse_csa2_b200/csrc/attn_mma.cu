@@ -461,11 +461,13 @@ struct AttnPlan {
 
 static bool use_tc_attention();
 
-static AttnPlan plan_attn(const csa_attn_args* a) {
+// `share`: how many attention launches of this size are expected to run at
+// the same time (concurrent layers of a stack); the SMs are divided among them.
+static AttnPlan plan_attn(const csa_attn_args* a, int share) {
   AttnPlan pl;
   const int n_entries = a->K + a->n_win;
   const int n_tiles = (n_entries + kTileE - 1) / kTileE;
-  const int64_t tokens = (int64_t)a->B * a->n_q;
+  const int64_t tokens = (int64_t)a->B * a->n_q * (share > 1 ? share : 1);
   int want = (int)((kNumSMs + tokens - 1) / tokens);
   // at least two tiles per split on the mma.sync kernel (each split reloads q
   // and writes a partial O); the tcgen05 kernel takes single tiles, its
@@ -479,8 +481,8 @@ static AttnPlan plan_attn(const csa_attn_args* a) {
   return pl;
 }
 
-size_t attn_ws_bytes(const csa_attn_args* a) {
-  AttnPlan pl = plan_attn(a);
+size_t attn_ws_bytes(const csa_attn_args* a, int share) {
+  AttnPlan pl = plan_attn(a, share);
   if (pl.n_splits <= 1) return 0;
   const size_t tok = (size_t)a->B * a->n_q;
   return tok * pl.n_splits * a->H * (kD + 2) * 4 + 256;
@@ -546,8 +548,8 @@ static cudaError_t launch_attn_64_tc(AttnParams& p, const void* q2, cudaStream_t
 // already staged by a layer stack's prologue).
 bool attn_tc_path(const csa_attn_args* a) { return a->H == 64 && use_tc_attention(); }
 
-cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2) {
-  AttnPlan pl = plan_attn(a);
+cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2, int share) {
+  AttnPlan pl = plan_attn(a, share);
   AttnParams p{};
   p.B = a->B; p.n_q = a->n_q; p.H = a->H;
   p.q = a->q;
