@@ -314,7 +314,9 @@ constexpr int kAuxStreams = 8;
 constexpr int kMaxStackLayers = 64;
 struct StackStreams {
   cudaStream_t aux[kAuxStreams] = {};
-  cudaEvent_t pro = nullptr;
+  cudaEvent_t start = nullptr;   // the caller's stream at the start of a step
+  cudaEvent_t pro = nullptr;     // prologue (appends, histogram clearing) done
+  cudaEvent_t stg = nullptr;     // decode queries staged
   cudaEvent_t idx[kMaxStackLayers] = {};
   cudaEvent_t done[kMaxStackLayers] = {};
   bool ok = false;
@@ -331,7 +333,9 @@ static StackStreams* stack_streams() {
     bool good = true;
     for (int i = 0; i < kAuxStreams && good; ++i)
       good = cudaStreamCreateWithFlags(&S.aux[i], cudaStreamNonBlocking) == cudaSuccess;
-    good = good && cudaEventCreateWithFlags(&S.pro, cudaEventDisableTiming) == cudaSuccess;
+    good = good && cudaEventCreateWithFlags(&S.pro, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&S.start, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&S.stg, cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < kMaxStackLayers && good; ++i)
       good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess &&
              cudaEventCreateWithFlags(&S.done[i], cudaEventDisableTiming) == cudaSuccess;
@@ -359,22 +363,25 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
   uint8_t* hist_base = base + w.layers;
   uint8_t* q2_base = hist_base + w.hists;
 
-  // prologue: every layer's appended rows, the clearing of every layer's
-  // histograms and the staging of decode queries, in one launch (each layer
-  // reads only rows appended before it in stream order, so moving the appends
-  // ahead of all layers is the same)
-  QuantBatch qb{};
+  // prologue on the caller's stream: every layer's appended rows and the
+  // clearing of every layer's histograms, in one launch (each layer reads only
+  // rows appended before it in stream order, so moving the appends ahead of
+  // all layers is the same).  The staging of the decode queries, which only
+  // the attention kernels read, runs on an auxiliary stream beside the first
+  // layer's scoring.
+  QuantBatch qb{}, qs{};
   qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
   qb.zero_n16 = (int64_t)(w.hists / 16);
-  auto add_job = [&](const void* src, int64_t n_rows, int64_t src_stride_bytes, void* dst, int64_t dst_stride,
-                     int fmt, int bf16, int dim) -> bool {
-    if (qb.njobs == kMaxBatchJobs) {
-      if (launch_quant_batch(qb, st) != cudaSuccess) return false;
-      qb.njobs = 0;
-      qb.units = 0;
-      qb.zero_n16 = 0;
+  cudaStream_t sst = SS->aux[kAuxStreams - 1];
+  auto add_job = [&](QuantBatch& q, cudaStream_t qs_stream, const void* src, int64_t n_rows,
+                     int64_t src_stride_bytes, void* dst, int64_t dst_stride, int fmt, int bf16, int dim) -> bool {
+    if (q.njobs == kMaxBatchJobs) {
+      if (launch_quant_batch(q, qs_stream) != cudaSuccess) return false;
+      q.njobs = 0;
+      q.units = 0;
+      q.zero_n16 = 0;
     }
-    QuantBatchJob& J = qb.job[qb.njobs++];
+    QuantBatchJob& J = q.job[q.njobs++];
     J.src = src;
     J.n_rows = n_rows;
     J.src_stride_bytes = src_stride_bytes;
@@ -383,17 +390,22 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     J.fmt = fmt;
     J.bf16 = bf16;
     J.dim = dim;
-    J.unit0 = qb.units;
-    qb.units += quant_batch_units(fmt, n_rows, dim);
+    J.unit0 = q.units;
+    q.units += quant_batch_units(fmt, n_rows, dim);
     return true;
   };
+  const bool staged = w.q2 > 0;
+  if (staged) {
+    if (cudaEventRecord(SS->start, st) != cudaSuccess || cudaStreamWaitEvent(sst, SS->start, 0) != cudaSuccess)
+      return CSA_ERR_CUDA;
+  }
   size_t q2_off = 0;
   for (int32_t i = 0; i < n_layers; ++i) {
     for (int k = 0; k < 3; ++k) {
       const csa_quant_job& q = layers[i].append[k];
       if (!q.src || q.n_rows == 0) continue;
       const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
-      if (!add_job(q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
+      if (!add_job(qb, st, q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
                    q.src_dtype == CSA_SRC_BF16, q.dim))
         return CSA_ERR_CUDA;
     }
@@ -401,13 +413,17 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     csa_attn_args at{};
     resolve_layer(layers, i, &ix, &at);
     if (layer_q2_bytes(at)) {
-      if (!add_job(at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
+      if (!add_job(qs, sst, at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
         return CSA_ERR_CUDA;
       q2_off += layer_q2_bytes(at);
     }
   }
   if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
   if (cudaEventRecord(SS->pro, st) != cudaSuccess) return CSA_ERR_CUDA;
+  if (staged) {
+    if (launch_quant_batch(qs, sst) != cudaSuccess) return CSA_ERR_CUDA;
+    if (cudaEventRecord(SS->stg, sst) != cudaSuccess) return CSA_ERR_CUDA;
+  }
 
   // Layers run concurrently where the mode stack allows it: layer 0 on the
   // caller's stream, layer i > 0 on an auxiliary stream that waits for the
@@ -437,6 +453,7 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
     const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
     q2_off += layer_q2_bytes(at);
+    if (q2 && cudaStreamWaitEvent(ls, SS->stg, 0) != cudaSuccess) return CSA_ERR_CUDA;
     if (run_sparse_attn(&at, region, ls, q2, share) != cudaSuccess) return CSA_ERR_CUDA;
     if (i > 0 && cudaEventRecord(SS->done[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
   }
