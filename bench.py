@@ -43,6 +43,24 @@ def _peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest value over all ranks; every rank calls it at the same point
+    (a device timing is reported as the slowest rank's)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: the tokens every rank decoded in one step over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_max * 1e-3)
+
+
 def _algorithmic_bytes(cfg):
     """HBM bytes a step must move (indexer keys + selected FP4 entries + window)."""
     per_layer_sel = cfg.B * cfg.K * 288
@@ -340,10 +358,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
     kernels = {k: (int(v[0]), float(v[1])) for k, v in kernels.items()}
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # ---- end to end through the public call: per-step inputs from pinned host
     # memory, the step, outputs back to pinned host memory
@@ -375,16 +390,12 @@ def run_gpu(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
     if rank != 0:
         return
     hbm_peak, _, peak_kind = _peaks()
-    tokens = cfg.B * world
-    value = tokens / (ms_max * 1e-3)
+    value = job_tokens_per_s(cfg.B, world, ms_max)
     alg = _algorithmic_bytes(cfg)
     # dominant kernel: the Full layer's indexer scoring over all T positions
     name = "index_score_tc[full]" if "index_score_tc[full]" in kernels else "index_score_decode[full]"
@@ -432,7 +443,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "kernels_note": f"from a second timed pass with an event pair around every kernel "
                         f"({round(profiled_ms, 4)} ms/step with the events)",
         "gpu_launches": int(launches),
-        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(cfg.B, world, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4)},
         "clocks": clk,
     }
