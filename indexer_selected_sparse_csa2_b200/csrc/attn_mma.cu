@@ -491,11 +491,9 @@ size_t attn_ws_bytes(const csa_attn_args* a, int share) {
 template <int H>
 static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes<H>();
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(sparse_attn_mma_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr = true;
-  }
+  static SmemAttrOnce attr;
+  const cudaError_t ea = attr.set(sparse_attn_mma_kernel<H>, smem);
+  if (ea != cudaSuccess) return ea;
   dim3 grid(p.n_splits, p.B * p.n_q);
   {
     ProfScope ps(stream, "sparse_attn_mma");

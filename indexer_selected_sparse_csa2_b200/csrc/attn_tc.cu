@@ -616,11 +616,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
 size_t attn_tc_smem_bytes() { return kAtSmemBytes; }
 
 cudaError_t launch_attn_tc(const AttnTcParams& p, cudaStream_t stream) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(sparse_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAtSmemBytes);
-    attr = true;
-  }
+  static SmemAttrOnce attr;
+  const cudaError_t ea = attr.set(sparse_attn_tc_kernel, kAtSmemBytes);
+  if (ea != cudaSuccess) return ea;
   dim3 grid(p.n_splits, p.B * p.n_q);
   ProfScope ps(stream, "sparse_attn_tc");
   launch_k(sparse_attn_tc_kernel, grid, dim3(kAtThreads), kAtSmemBytes, stream, p);

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
+#include <atomic>
 #include <utility>
 
 #include "../../include/csa.h"
@@ -110,6 +111,28 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+// A kernel's dynamic shared-memory limit, raised once per device:
+// cudaFuncSetAttribute applies to the current device only, so a process that
+// drives several GPUs must set it on each.  Thread-safe (a race sets it twice,
+// which is harmless).
+class SmemAttrOnce {
+ public:
+  template <typename... KArgs>
+  cudaError_t set(void (*kernel)(KArgs...), size_t bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t)1 << dev : 0;
+    if (bit && (done_.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && bit) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
 
 // Host-side launch accounting (see csa_launch_count()) and opt-in event
 // timing of each launch (see csa_profile_enable()).

@@ -656,14 +656,10 @@ cudaError_t run_index_prefill(const csa_index_args* a, void* ws, cudaStream_t st
   e = launch_zero(w.sel.hist, (size_t)rows * kHistBins * 4, stream);
   if (e != cudaSuccess) return e;
 
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(prefill_score_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmemBytes);
-    cudaFuncSetAttribute(prefill_score_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPfSmemBytes);
-    cudaFuncSetAttribute(prefill_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)((2 * kCandCap + 2 * kPfMaxK) * 4));
-    attr = true;
-  }
+  static SmemAttrOnce attr0, attr1, attr_final;
+  if ((e = attr0.set(prefill_score_tc_kernel<0>, kPfSmemBytes)) != cudaSuccess) return e;
+  if ((e = attr1.set(prefill_score_tc_kernel<1>, kPfSmemBytes)) != cudaSuccess) return e;
+  if ((e = attr_final.set(prefill_final_kernel, (size_t)(2 * kCandCap + 2 * kPfMaxK) * 4)) != cudaSuccess) return e;
   PfParams p{};
   p.q = a->q;
   p.w = a->w;

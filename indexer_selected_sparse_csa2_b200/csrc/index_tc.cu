@@ -247,11 +247,9 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
   p.bhist = bhist;
   p.nb = nb;
   p.block_len = a->pool_block_len;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(index_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmemBytes);
-    attr = true;
-  }
+  static SmemAttrOnce attr;
+  const cudaError_t ea = attr.set(index_score_tc_kernel, kTcSmemBytes);
+  if (ea != cudaSuccess) return ea;
   ProfScope ps(stream, "index_score_tc[full]");
   launch_k(index_score_tc_kernel, dim3(dim3((unsigned)ctas_row, (unsigned)a->B)), dim3(kTcThreads), kTcSmemBytes, stream, map, p);
   note_launches(1);

@@ -585,11 +585,9 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
     else launch_k(select_extract_kernel<false>, dim3(g), dim3(kExtractThreads), 0, stream, js);
   }
   const size_t smem = (size_t)kMaxRuns * 4 + (size_t)kListCap * 8;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    attr_set = true;
-  }
+  static SmemAttrOnce attr;
+  const cudaError_t ea = attr.set(select_final_kernel, smem);
+  if (ea != cudaSuccess) return ea;
   {
     ProfScope ps(stream, "select_final");
     launch_k(select_final_kernel, dim3(dim3(B, njobs)), dim3(kFinalThreads), smem, stream, js);
