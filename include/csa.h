@@ -30,7 +30,9 @@
  *     returns a non-zero csa_status and enqueues nothing.  A failed launch
  *     returns CSA_ERR_CUDA.
  *   - Byte strides and entry pointers must be 16-byte aligned.
- *   - Calls keep no state between them and may be captured in a CUDA graph.
+ *   - Calls keep no device state between them and may be captured in a
+ *     CUDA graph (csa_layer_step keeps host-side streams and events per
+ *     device; see there).
  */
 #ifndef CSA_H_
 #define CSA_H_
@@ -196,7 +198,7 @@ csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t works
                            csa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* A stack of layers run in order on one stream.
+/* A stack of layers, one decode (or prefill) step.
  *   FULL    : encode `append` rows, index.* scoring + Top-K (+ pool build),
  *             then attention with attn.idx = index.idx.
  *   REINDEX : as FULL (index.keys and attn.kv normally point at the owner
@@ -205,7 +207,18 @@ csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t works
  *   REUSE   : no scoring; attention with attn.idx = the idx of layer
  *             reuse_from (attn.K likewise).
  * `append[i]` with src != NULL encodes new rows (e.g. this step's token)
- * into the caches before the layer's scoring. */
+ * into the caches before any layer's scoring (all appends of the stack run
+ * first, in one launch).
+ *
+ * Ordering: the result is as if the layers ran in order on `stream`.
+ * Internally, layers that do not depend on each other run concurrently on
+ * auxiliary streams that the library creates once per device (no device
+ * memory). Each auxiliary stream forks from `stream` by event and is joined
+ * back into `stream` before the call returns, also when a launch fails part
+ * way. Work enqueued on `stream` afterwards therefore sees every output, and
+ * a stream capture of the call records the fork and join as graph edges.
+ * Calls from several host threads are allowed: enqueues on one device are
+ * serialised by a lock. */
 typedef struct {
   const void* src;           /* NULL = no job */
   int32_t src_dtype;

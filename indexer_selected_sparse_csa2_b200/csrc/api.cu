@@ -318,7 +318,8 @@ struct StackStreams {
   cudaEvent_t pro = nullptr;     // prologue (appends, histogram clearing) done
   cudaEvent_t stg = nullptr;     // decode queries staged
   cudaEvent_t idx[kMaxStackLayers] = {};
-  cudaEvent_t done[kMaxStackLayers] = {};
+  cudaEvent_t join[kAuxStreams] = {};   // tail of an auxiliary stream, joined into the caller's
+  std::mutex mu;                        // one step enqueues on this device's streams at a time
   bool ok = false;
 };
 static std::mutex g_stack_mu;
@@ -337,8 +338,9 @@ static StackStreams* stack_streams() {
            cudaEventCreateWithFlags(&S.start, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&S.stg, cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < kMaxStackLayers && good; ++i)
-      good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&S.done[i], cudaEventDisableTiming) == cudaSuccess;
+      good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < kAuxStreams && good; ++i)
+      good = cudaEventCreateWithFlags(&S.join[i], cudaEventDisableTiming) == cudaSuccess;
     if (!good) return nullptr;
     S.ok = true;
   }
@@ -359,107 +361,120 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
   StackStreams* SS = stack_streams();
   if (!SS) return CSA_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint8_t* hist_base = base + w.layers;
-  uint8_t* q2_base = hist_base + w.hists;
+  // The step enqueues on library-owned auxiliary streams and events of this
+  // device: one caller at a time, and every auxiliary stream it used is
+  // joined into the caller's stream again, also when a launch fails half way.
+  std::lock_guard<std::mutex> lk(SS->mu);
+  bool used[kAuxStreams] = {};
+  auto enqueue = [&]() -> csa_status {
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    uint8_t* hist_base = base + w.layers;
+    uint8_t* q2_base = hist_base + w.hists;
 
-  // prologue on the caller's stream: every layer's appended rows and the
-  // clearing of every layer's histograms, in one launch (each layer reads only
-  // rows appended before it in stream order, so moving the appends ahead of
-  // all layers is the same).  The staging of the decode queries, which only
-  // the attention kernels read, runs on an auxiliary stream beside the first
-  // layer's scoring.
-  QuantBatch qb{}, qs{};
-  qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
-  qb.zero_n16 = (int64_t)(w.hists / 16);
-  cudaStream_t sst = SS->aux[kAuxStreams - 1];
-  auto add_job = [&](QuantBatch& q, cudaStream_t qs_stream, const void* src, int64_t n_rows,
-                     int64_t src_stride_bytes, void* dst, int64_t dst_stride, int fmt, int bf16, int dim) -> bool {
-    if (q.njobs == kMaxBatchJobs) {
-      if (launch_quant_batch(q, qs_stream) != cudaSuccess) return false;
-      q.njobs = 0;
-      q.units = 0;
-      q.zero_n16 = 0;
-    }
-    QuantBatchJob& J = q.job[q.njobs++];
-    J.src = src;
-    J.n_rows = n_rows;
-    J.src_stride_bytes = src_stride_bytes;
-    J.dst = static_cast<uint8_t*>(dst);
-    J.dst_stride = dst_stride;
-    J.fmt = fmt;
-    J.bf16 = bf16;
-    J.dim = dim;
-    J.unit0 = q.units;
-    q.units += quant_batch_units(fmt, n_rows, dim);
-    return true;
-  };
-  const bool staged = w.q2 > 0;
-  if (staged) {
-    if (cudaEventRecord(SS->start, st) != cudaSuccess || cudaStreamWaitEvent(sst, SS->start, 0) != cudaSuccess)
-      return CSA_ERR_CUDA;
-  }
-  size_t q2_off = 0;
-  for (int32_t i = 0; i < n_layers; ++i) {
-    for (int k = 0; k < 3; ++k) {
-      const csa_quant_job& q = layers[i].append[k];
-      if (!q.src || q.n_rows == 0) continue;
-      const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
-      if (!add_job(qb, st, q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
-                   q.src_dtype == CSA_SRC_BF16, q.dim))
+    // prologue on the caller's stream: every layer's appended rows and the
+    // clearing of every layer's histograms, in one launch (each layer reads only
+    // rows appended before it in stream order, so moving the appends ahead of
+    // all layers is the same).  The staging of the decode queries, which only
+    // the attention kernels read, runs on an auxiliary stream beside the first
+    // layer's scoring.
+    QuantBatch qb{}, qs{};
+    qb.zero_ptr = reinterpret_cast<uint4*>(hist_base);
+    qb.zero_n16 = (int64_t)(w.hists / 16);
+    cudaStream_t sst = SS->aux[kAuxStreams - 1];
+    auto add_job = [&](QuantBatch& q, cudaStream_t qs_stream, const void* src, int64_t n_rows,
+                       int64_t src_stride_bytes, void* dst, int64_t dst_stride, int fmt, int bf16, int dim) -> bool {
+      if (q.njobs == kMaxBatchJobs) {
+        if (launch_quant_batch(q, qs_stream) != cudaSuccess) return false;
+        q.njobs = 0;
+        q.units = 0;
+        q.zero_n16 = 0;
+      }
+      QuantBatchJob& J = q.job[q.njobs++];
+      J.src = src;
+      J.n_rows = n_rows;
+      J.src_stride_bytes = src_stride_bytes;
+      J.dst = static_cast<uint8_t*>(dst);
+      J.dst_stride = dst_stride;
+      J.fmt = fmt;
+      J.bf16 = bf16;
+      J.dim = dim;
+      J.unit0 = q.units;
+      q.units += quant_batch_units(fmt, n_rows, dim);
+      return true;
+    };
+    const bool staged = w.q2 > 0;
+    if (staged) {
+      used[kAuxStreams - 1] = true;
+      if (cudaEventRecord(SS->start, st) != cudaSuccess || cudaStreamWaitEvent(sst, SS->start, 0) != cudaSuccess)
         return CSA_ERR_CUDA;
     }
-    csa_index_args ix{};
-    csa_attn_args at{};
-    resolve_layer(layers, i, &ix, &at);
-    if (layer_q2_bytes(at)) {
-      if (!add_job(qs, sst, at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
+    size_t q2_off = 0;
+    for (int32_t i = 0; i < n_layers; ++i) {
+      for (int k = 0; k < 3; ++k) {
+        const csa_quant_job& q = layers[i].append[k];
+        if (!q.src || q.n_rows == 0) continue;
+        const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
+        if (!add_job(qb, st, q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
+                     q.src_dtype == CSA_SRC_BF16, q.dim))
+          return CSA_ERR_CUDA;
+      }
+      csa_index_args ix{};
+      csa_attn_args at{};
+      resolve_layer(layers, i, &ix, &at);
+      if (layer_q2_bytes(at)) {
+        if (!add_job(qs, sst, at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
+          return CSA_ERR_CUDA;
+        q2_off += layer_q2_bytes(at);
+      }
+    }
+    if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
+    if (cudaEventRecord(SS->pro, st) != cudaSuccess) return CSA_ERR_CUDA;
+    if (staged) {
+      if (launch_quant_batch(qs, sst) != cudaSuccess) return CSA_ERR_CUDA;
+      if (cudaEventRecord(SS->stg, sst) != cudaSuccess) return CSA_ERR_CUDA;
+    }
+
+    // Layers run concurrently where the mode stack allows it: layer 0 on the
+    // caller's stream, layer i > 0 on an auxiliary stream that waits for the
+    // prologue, for the pool builder's Top-K (Reindex in a pool) or for the
+    // reused layer's Top-K (Reuse); the caller's stream then waits for all.
+    size_t reg_off = 0, hist_off = 0;
+    q2_off = 0;
+    for (int32_t i = 0; i < n_layers; ++i) {
+      csa_index_args ix{};
+      csa_attn_args at{};
+      resolve_layer(layers, i, &ix, &at);
+      const csa_layer_desc& L = layers[i];
+      if (i > 0) used[(i - 1) % kAuxStreams] = true;
+      cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kAuxStreams];
+      if (i > 0 && cudaStreamWaitEvent(ls, SS->pro, 0) != cudaSuccess) return CSA_ERR_CUDA;
+      uint8_t* region = base + reg_off;
+      const int share = attn_share(layers, n_layers, i);
+      reg_off += layer_region_bytes(L, ix, at, share);
+      if (L.mode != CSA_MODE_REUSE) {
+        if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->idx[L.pool_from], 0) != cudaSuccess)
+          return CSA_ERR_CUDA;
+        uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
+        hist_off += index_hist_bytes(&ix);
+        if (run_index_decode(&ix, region, ls, h) != cudaSuccess) return CSA_ERR_CUDA;
+      } else if (cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
         return CSA_ERR_CUDA;
+      }
+      if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
+      const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
       q2_off += layer_q2_bytes(at);
+      if (q2 && cudaStreamWaitEvent(ls, SS->stg, 0) != cudaSuccess) return CSA_ERR_CUDA;
+      if (run_sparse_attn(&at, region, ls, q2, share) != cudaSuccess) return CSA_ERR_CUDA;
     }
-  }
-  if (launch_quant_batch(qb, st) != cudaSuccess) return CSA_ERR_CUDA;
-  if (cudaEventRecord(SS->pro, st) != cudaSuccess) return CSA_ERR_CUDA;
-  if (staged) {
-    if (launch_quant_batch(qs, sst) != cudaSuccess) return CSA_ERR_CUDA;
-    if (cudaEventRecord(SS->stg, sst) != cudaSuccess) return CSA_ERR_CUDA;
-  }
-
-  // Layers run concurrently where the mode stack allows it: layer 0 on the
-  // caller's stream, layer i > 0 on an auxiliary stream that waits for the
-  // prologue, for the pool builder's Top-K (Reindex in a pool) or for the
-  // reused layer's Top-K (Reuse); the caller's stream then waits for all.
-  size_t reg_off = 0, hist_off = 0;
-  q2_off = 0;
-  for (int32_t i = 0; i < n_layers; ++i) {
-    csa_index_args ix{};
-    csa_attn_args at{};
-    resolve_layer(layers, i, &ix, &at);
-    const csa_layer_desc& L = layers[i];
-    cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kAuxStreams];
-    if (i > 0 && cudaStreamWaitEvent(ls, SS->pro, 0) != cudaSuccess) return CSA_ERR_CUDA;
-    uint8_t* region = base + reg_off;
-    const int share = attn_share(layers, n_layers, i);
-    reg_off += layer_region_bytes(L, ix, at, share);
-    if (L.mode != CSA_MODE_REUSE) {
-      if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->idx[L.pool_from], 0) != cudaSuccess)
-        return CSA_ERR_CUDA;
-      uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
-      hist_off += index_hist_bytes(&ix);
-      if (run_index_decode(&ix, region, ls, h) != cudaSuccess) return CSA_ERR_CUDA;
-    } else if (cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
+    return CSA_OK;
+  };
+  const csa_status rc = enqueue();
+  for (int k = 0; k < kAuxStreams; ++k) {
+    if (!used[k]) continue;
+    if (cudaEventRecord(SS->join[k], SS->aux[k]) != cudaSuccess || cudaStreamWaitEvent(st, SS->join[k], 0) != cudaSuccess)
       return CSA_ERR_CUDA;
-    }
-    if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
-    const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
-    q2_off += layer_q2_bytes(at);
-    if (q2 && cudaStreamWaitEvent(ls, SS->stg, 0) != cudaSuccess) return CSA_ERR_CUDA;
-    if (run_sparse_attn(&at, region, ls, q2, share) != cudaSuccess) return CSA_ERR_CUDA;
-    if (i > 0 && cudaEventRecord(SS->done[i], ls) != cudaSuccess) return CSA_ERR_CUDA;
   }
-  for (int32_t i = 1; i < n_layers; ++i)
-    if (cudaStreamWaitEvent(st, SS->done[i], 0) != cudaSuccess) return CSA_ERR_CUDA;
-  return CSA_OK;
+  return rc;
 }
 
 const char* csa_status_string(int32_t s) {
