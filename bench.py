@@ -383,7 +383,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
         e_starts[i].record(stream)
         for h, d in h2d_pairs:
             d.copy_(h, non_blocking=True)
-        run_step()
+        step()                      # the C-ABI call itself, launched eagerly
         for h, d in d2h_pairs:
             h.copy_(d, non_blocking=True)
         e_ends[i].record(stream)
@@ -444,7 +444,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
                         f"({round(profiled_ms, 4)} ms/step with the events)",
         "gpu_launches": int(launches),
         "e2e": {"value": round(job_tokens_per_s(cfg.B, world, e2e_ms), 2), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4)},
+                "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4),
+                "path": "csa_layer_step called through the Python binding each step (no graph), "
+                        "pinned host inputs copied in and outputs copied back inside the timed events"},
         "clocks": clk,
     }
     if world == 1 and not args.no_prefill:
