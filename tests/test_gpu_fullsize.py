@@ -66,21 +66,52 @@ def _compare_layers(cfg, dc, b, res, queries, t_index):
     assert n_identical >= 0.75 * n_rows, (n_identical, n_rows)
 
 
-def _run_decode(csa, name, batches):
+def _clear_outputs(dc):
+    for dl in dc.layers:
+        dl.out.zero_()
+        dl.lse.zero_()
+        dl.idx.fill_(-7)
+        if dl.pool is not None:
+            dl.pool.fill_(-7)
+            dl.pool_len.zero_()
+
+
+def _run_decode(csa, name, batches, graph=False):
+    """The step eagerly; with `graph`, then also captured into a CUDA graph on
+    a side stream and replayed, as the benchmark times it (outputs cleared
+    before the replay), both checked against the same oracle results."""
     from csa_synth.device import DeviceCase
     cfg = get_config(name)
     dc = DeviceCase(cfg, keep_scores=False)
-    csa.csa_layer_step(dc.layer_descs(append_rows=True))
+    descs = dc.layer_descs(append_rows=True)
+    ws = torch.empty(max(csa.csa_layer_workspace_size(descs), 16), dtype=torch.uint8, device="cuda")
+    csa.csa_layer_step(descs, workspace=ws)
     torch.cuda.synchronize()
     assert csa.device_status() == 0
+    results = {}
     for b in batches:
         case = SynthCase(cfg, b, threads=os.cpu_count() or 4, dense_latents=True)
         for o in cfg.owners:
             rows = np.array([0, 1, cfg.T // 2, cfg.T - 1])
             assert np.array_equal(dc.keys[o][b].cpu().numpy()[rows], case.keys(o)[rows])
             assert np.array_equal(dc.kv[o][b, torch.from_numpy(rows)].cpu().numpy(), case.main_entries(o, rows))
-        res = case.run(keep_scores=True)
-        _compare_layers(cfg, dc, b, res, [0], None)
+        results[b] = case.run(keep_scores=True)
+        _compare_layers(cfg, dc, b, results[b], [0], None)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cap):
+            csa.csa_layer_step(descs, workspace=ws, stream=cap)
+        torch.cuda.synchronize()
+        _clear_outputs(dc)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert csa.device_status() == 0
+        for b in batches:
+            _compare_layers(cfg, dc, b, results[b], [0], None)
+        del g
 
 
 def test_fullsize_tiny_decode(csa):
@@ -96,7 +127,7 @@ def test_fullsize_stack_128k(csa):
 
 
 def test_fullsize_hier_1m(csa):
-    _run_decode(csa, "hier_1m", [0, 3])
+    _run_decode(csa, "hier_1m", [0, 3], graph=True)
 
 
 def test_fullsize_prefill_1m(csa):
