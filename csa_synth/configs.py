@@ -55,6 +55,7 @@ class Config:
     planted: bool = False     # planted high-score keys every ~4096 positions
     plant_stride: int = 4096
     bf16_latents: bool = False
+    key_format: str = "e4m3"  # indexer keys: "e4m3" (plain cast) or "mxfp4" (E2M1 + E8M0 per 32)
 
     @property
     def softmax_scale(self) -> float:
@@ -94,6 +95,10 @@ CONFIGS = {
                 LayerSpec(REINDEX, 0, pool_from=0)]),
     "prefill_1m": Config(name="prefill_1m", B=1, T=1 << 20, H=64, H_I=8, K=2048, seed=4,
                          n_q=4096, bf16_latents=True),
+    # the pages' own indexer shape and key format (32 heads x 128, MXFP4 keys
+    # of 68 B, top-512): the oracle side of the next row of the scope table
+    "decode_mx": Config(name="decode_mx", B=8, T=65536, H=64, H_I=32, K=512, seed=5, d_I=128,
+                        key_format="mxfp4"),
     # a quarter-size prefill chunk (profiling captures that must stay small)
     "prefill_256k": Config(name="prefill_256k", B=1, T=1 << 18, H=64, H_I=8, K=2048, seed=4,
                            n_q=1024, bf16_latents=True),

@@ -46,6 +46,8 @@ class DeviceCase:
                  keep_scores: bool = False, batches: Optional[List[int]] = None):
         import torch
         csa = _lib()
+        if cfg.key_format != "e4m3":
+            raise NotImplementedError(f"indexer key format {cfg.key_format!r} has no device encoder")
         self.cfg = cfg
         self.device = device
         B, T = cfg.B, cfg.T

@@ -14,6 +14,7 @@ from csa_synth import workload as wl
 from csa_synth.configs import Config
 
 from .quant import fp4_quant_rows, fp8_window_quant_rows, e4m3_cast
+from .mxfp4 import mxfp4_quant_rows
 from .layers import LayerInputs, run_stack
 
 
@@ -33,7 +34,7 @@ class SynthCase:
     def keys(self, owner: int) -> np.ndarray:
         if owner not in self._keys:
             x = wl.index_key(self.cfg, owner, self.b, 0, self.cfg.T, threads=self.threads)
-            self._keys[owner] = e4m3_cast(x)
+            self._keys[owner] = mxfp4_quant_rows(x) if self.cfg.key_format == "mxfp4" else e4m3_cast(x)
         return self._keys[owner]
 
     def main_entries(self, owner: int, positions: np.ndarray) -> np.ndarray:
@@ -61,4 +62,4 @@ class SynthCase:
         return run_stack(c.layers, c.T, c.n_q, c.K, c.n_win, c.softmax_scale,
                          self.keys, self.main_entries, self.inputs, queries=queries,
                          pool_blocks=c.pool_blocks, pool_block_len=c.pool_block_len,
-                         keep_scores=keep_scores)
+                         keep_scores=keep_scores, key_format=c.key_format)

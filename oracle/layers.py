@@ -28,6 +28,7 @@ from typing import Callable, Dict, List, Optional, Sequence
 import numpy as np
 
 from .indexer import index_scores, topk, build_pool
+from .mxfp4 import mx_index_scores
 from .attention import attend
 from .quant import fp4_dequant_rows, fp8_window_dequant_rows
 
@@ -60,16 +61,18 @@ def run_stack(layers: Sequence, T: int, n_q: int, K: int, n_win: int, scale: flo
               inputs: Callable[[int], LayerInputs],
               queries: Optional[Sequence[int]] = None,
               pool_blocks: int = 2048, pool_block_len: int = 8,
-              keep_scores: bool = False) -> List[LayerResult]:
+              keep_scores: bool = False, key_format: str = "e4m3") -> List[LayerResult]:
     """Run a layer stack for one sequence.
 
     ``layers``: objects with mode / owner / reuse_from / build_pool / pool_from.
-    ``keys(owner)``: uint8 [T, d_I] indexer key codes of the owner layer.
+    ``keys(owner)``: uint8 indexer keys of the owner layer: [T, d_I] E4M3 codes,
+    or [T, d_I/2 + d_I/32] MXFP4 entries when ``key_format`` is "mxfp4".
     ``main_entries(owner, positions)``: uint8 [n, 288] main-KV entries.
     ``inputs(layer)``: that layer's LayerInputs.
     ``queries``: query token indices to evaluate (default all n_q).
     """
     qs = list(range(n_q)) if queries is None else list(queries)
+    score = mx_index_scores if key_format == "mxfp4" else index_scores
     results: List[LayerResult] = []
     for li, L in enumerate(layers):
         inp = inputs(li)
@@ -85,10 +88,10 @@ def run_stack(layers: Sequence, T: int, n_q: int, K: int, n_win: int, scale: flo
                 if L.mode == REINDEX and L.pool_from >= 0:
                     P = results[L.pool_from]
                     ppos = P.pool[:P.pool_len].astype(np.int64)
-                    S = index_scores(inp.qI[t], inp.w[t], kc[ppos])
+                    S = score(inp.qI[t], inp.w[t], kc[ppos])
                     idx_rows.append(topk(S, K, ppos))
                 else:
-                    S = index_scores(inp.qI[t], inp.w[t], kc[:n_t])
+                    S = score(inp.qI[t], inp.w[t], kc[:n_t])
                     idx_rows.append(topk(S, K))
                     if L.build_pool:
                         pool, pool_len = build_pool(S, pool_blocks, pool_block_len)

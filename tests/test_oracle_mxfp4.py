@@ -179,3 +179,29 @@ def test_equals_plain_e4m3_keys_when_both_represent_them():
     assert np.array_equal(mx.mxfp4_dequant_rows(entries), k.astype(np.float64))
     assert np.array_equal(mx.mx_index_scores(q_codes, w, entries),
                           indexer.index_scores(q_codes, w, quant.e4m3_cast(k)))
+
+
+def test_stack_with_mxfp4_keys_end_to_end():
+    """The oracle's stack run on the pages' indexer shape (32 heads x 128,
+    MXFP4 keys, top-512) equals the pieces composed by hand: MXFP4 entries of
+    the seeded keys, their scores, the Top-K and the attention over it."""
+    from csa_synth import get_config
+    from csa_synth import workload as wl
+    from oracle.case import SynthCase
+    from oracle.attention import attend
+    cfg = get_config("decode_mx", B=1, T=3000)
+    case = SynthCase(cfg, 0)
+    keys = case.keys(0)
+    assert keys.shape == (cfg.T, 68)
+    assert np.array_equal(keys, mx.mxfp4_quant_rows(wl.index_key(cfg, 0, 0, 0, cfg.T)))
+    res = case.run(keep_scores=True)[0]
+    inp = case.inputs(0)
+    assert inp.qI.shape == (1, 32, 128)
+    S = mx.mx_index_scores(inp.qI[0], inp.w[0], keys)
+    assert np.array_equal(res.scores[0], S)
+    assert np.array_equal(res.idx[0], indexer.topk(S, 512))
+    sel = res.idx[0][res.idx[0] >= 0].astype(np.int64)
+    X = np.concatenate([quant.fp4_dequant_rows(case.main_entries(0, sel)),
+                        quant.fp8_window_dequant_rows(inp.window[0:cfg.n_win])])
+    o, l = attend(inp.q[0], X, cfg.softmax_scale, None)
+    assert np.array_equal(res.out[0], o) and np.array_equal(res.lse[0], l)
