@@ -240,9 +240,9 @@ def csa_attn_workspace_size(args: AttnArgs) -> int:
 
 
 def csa_sparse_attn(args: AttnArgs, workspace=None, stream=None, device=None) -> None:
-    need = csa_attn_workspace_size(args)
+    # the library checks a given workspace's size itself; query it only to allocate one
     if workspace is None:
-        workspace = _workspace(need, device or "cuda")
+        workspace = _workspace(csa_attn_workspace_size(args), device or "cuda")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_attn(ctypes.byref(args), _ptr(workspace), nbytes, _stream(stream)), "csa_sparse_attn")
 
@@ -264,9 +264,9 @@ def csa_layer_workspace_size(layers) -> int:
 
 def csa_layer_step(layers, workspace=None, stream=None, device=None) -> None:
     """Run a ctypes array of LayerDesc (see ``make_layer_array``) on one stream."""
-    need = csa_layer_workspace_size(layers)
+    # the library checks a given workspace's size itself; query it only to allocate one
     if workspace is None:
-        workspace = _workspace(need, device or "cuda")
+        workspace = _workspace(csa_layer_workspace_size(layers), device or "cuda")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_layer(layers, len(layers), _ptr(workspace), nbytes, _stream(stream)), "csa_layer_step")
 
