@@ -34,13 +34,82 @@ FLUSH_BYTES = 256 << 20          # > 126 MB L2
 L2_BYTES = 126 << 20
 
 
-def _peaks():
+def _file_peaks():
+    """The machine's measured peaks (context beside the in-run ones), else
+    the recipe's fallback figures."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "kind": "measured (file)"}
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "kind": "fallback"}
+
+
+def _time_ms(fn, reps, stream):
+    """Best CUDA-event time of `reps` calls (after two untimed calls)."""
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        best = min(best, a.elapsed_time(b))
+    return best
+
+
+def measure_peaks(dev):
+    """The roofline denominators, measured in this run on this GPU:
+    * hbm_gbs: the library's 128-bit copy kernel over 2 GiB (read + write);
+    * fp8_tflops: the library's tcgen05 FP8 GEMM at 8192^3, cross-checked
+      with cuBLAS FP8 (torch._scaled_mm); the larger of the two is the peak;
+    * bf16_tflops: cuBLAS bf16 GEMM at 8192^3 (torch.matmul)."""
+    import torch
+    import indexer_selected_sparse_csa2_b200 as csa
+    stream = torch.cuda.current_stream()
+    out = {}
+    n = 2 << 30
+    src = torch.empty(n, dtype=torch.uint8, device=dev)
+    dst = torch.empty(n, dtype=torch.uint8, device=dev)
+    src.fill_(7)
+    ms = _time_ms(lambda: csa.csa_bench_copy(src, dst, stream=stream), 10, stream)
+    out["hbm_gbs"] = round(2 * n / (ms * 1e-3) / 1e9, 1)
+    out["copy_bytes"] = 2 * n
+    del src, dst
+    S = 8192
+    g = torch.Generator(device=dev).manual_seed(5)
+    A = torch.randint(0, 126, (S, S), dtype=torch.uint8, device=dev, generator=g)   # finite E4M3 codes
+    B = torch.randint(0, 126, (S, S), dtype=torch.uint8, device=dev, generator=g)
+    D = torch.empty(S, S, dtype=torch.float32, device=dev)
+    flops = 2.0 * S ** 3
+    ms = _time_ms(lambda: csa.csa_bench_fp8_gemm(A, B, D, stream=stream), 5, stream)
+    own = flops / (ms * 1e-3) / 1e12
+    out["fp8_own_tflops"] = round(own, 1)
+    try:
+        a8 = A.view(torch.float8_e4m3fn)
+        b8 = B.view(torch.float8_e4m3fn)
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        ms_c = _time_ms(lambda: torch._scaled_mm(a8, b8.t(), scale_a=one, scale_b=one,
+                                                 out_dtype=torch.bfloat16), 5, stream)
+        out["fp8_cublas_tflops"] = round(flops / (ms_c * 1e-3) / 1e12, 1)
+    except Exception as e:       # cross-check only
+        out["fp8_cublas_error"] = repr(e)[:120]
+    out["fp8_tflops"] = max(out["fp8_own_tflops"], out.get("fp8_cublas_tflops", 0.0))
+    del A, B, D
+    x = torch.randn(S, S, dtype=torch.bfloat16, device=dev)
+    y = torch.randn(S, S, dtype=torch.bfloat16, device=dev)
+    ms = _time_ms(lambda: torch.matmul(x, y), 5, stream)
+    out["bf16_tflops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    del x, y
+    torch.cuda.empty_cache()
+    out["kind"] = "measured in this run (burst: kernels timed alone)"
+    out["file"] = _file_peaks()
+    return out
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
@@ -76,19 +145,86 @@ def _algorithmic_bytes(cfg):
     return keys + len(cfg.layers) * (per_layer_sel + per_layer_win)
 
 
-def _traffic_record(kernel_src):
-    """(bytes per launch, sha) from the committed ncu summary, if it matches the source."""
-    path = os.path.join(ROOT, "profiles", "index_score_decode_hier_1m.md")
-    try:
+KERNEL_SOURCES = {
+    "index_score_tc[full]": "index_tc.cu",
+    "index_score_decode[pool]": "index_decode.cu",
+    "sparse_attn_tc": "attn_tc.cu",
+    "attn_combine": "attn_mma.cu",
+    "select_extract": "select.cu",
+    "select_final": "select.cu",
+    "select_small": "select.cu",
+    "quant_batch": "quant.cu",
+}
+
+
+def _traffic_record(kernel):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary under
+    profiles/ ("bench_kernel: <name>", "traffic_bytes_per_launch: <n>",
+    "kernel_source_sha1: <sha>"), only while that kernel's source file still
+    has the recorded sha1; else None."""
+    import glob
+    src = KERNEL_SOURCES.get(kernel)
+    if not src:
+        return None
+    sha = hashlib.sha1(open(os.path.join(ROOT, "indexer_selected_sparse_csa2_b200", "csrc", src), "rb")
+                       .read()).hexdigest()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         txt = open(path).read()
-    except OSError:
-        return None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
-    h = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", txt)
-    if not m or not h:
-        return None
-    sha = hashlib.sha1(open(kernel_src, "rb").read()).hexdigest()
-    return int(m.group(1)) if h.group(1) == sha else None
+        for blk in txt.split("bench_kernel:")[1:]:
+            name = blk.split()[0]
+            m = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", blk)
+            h = re.search(r"kernel_source_sha1:\s*([0-9a-f]+)", blk)
+            if name == kernel and m and h and h.group(1) == sha:
+                return int(m.group(1))
+    return None
+
+
+def kernel_work(cfg):
+    """Algorithmic HBM bytes and flops per launch of the decode step's kernels
+    (what the kernel must read or write, and the multiply-adds x 2 it must do):
+    * full scorer: B*T keys of 64 B; 2*64*H_I flops per (key, head);
+    * pool scorer: B*pool keys of 64 B (one Reindex layer per launch);
+    * attention: B*(K*288 + W*528) entry bytes; 2 * 2*H*512 flops per entry
+      (logits and the weighted sum), one layer per launch;
+    * selects and the split combine: the scores / partials they read."""
+    B, T, K, W, H, HI = cfg.B, cfg.T, cfg.K, cfg.n_win, cfg.H, cfg.H_I
+    n_pool = cfg.pool_blocks * cfg.pool_block_len
+    return {
+        "index_score_tc[full]": {"bytes": B * T * 64, "flops": 2.0 * B * T * HI * 64, "engine": "fp8"},
+        "index_score_decode[pool]": {"bytes": B * n_pool * 64, "flops": 2.0 * B * n_pool * HI * 64, "engine": "fp8"},
+        "sparse_attn_tc": {"bytes": B * (K * 288 + W * 528), "flops": 4.0 * B * H * 512 * (K + W), "engine": "bf16"},
+        "select_extract": {"bytes": B * T * 4, "flops": 0.0, "engine": None},
+        "select_small": {"bytes": B * n_pool * 4, "flops": 0.0, "engine": None},
+    }
+
+
+def roofline_of(name, work, ms_launch, peaks, traffic):
+    """Roofline record of one kernel: achieved bytes/s and flops/s against the
+    measured HBM and tensor peaks; `bound` is the roof it is nearer to."""
+    w = work.get(name)
+    if not w or not ms_launch or ms_launch != ms_launch:
+        return {"kernel": name, "launch_ms": ms_launch, "bound": None, "achieved": None, "peak": None,
+                "unit": None, "frac": None, "traffic": traffic, "note": "no algorithmic work recorded"}
+    gbs = w["bytes"] / (ms_launch * 1e-3) / 1e9
+    hbm_frac = gbs / peaks["hbm_gbs"]
+    rec = {"kernel": name, "launch_ms": round(ms_launch, 5), "bytes_per_launch": w["bytes"],
+           "flops_per_launch": w["flops"], "hbm_gbs": round(gbs, 1), "hbm_frac": round(hbm_frac, 4)}
+    t_frac = None
+    if w["engine"]:
+        tpeak = peaks["fp8_tflops"] if w["engine"] == "fp8" else peaks["bf16_tflops"]
+        tfl = w["flops"] / (ms_launch * 1e-3) / 1e12
+        t_frac = tfl / tpeak
+        rec.update({"tflops": round(tfl, 2), "tensor_peak": tpeak, "tensor_frac": round(t_frac, 4),
+                    "tensor_peak_kind": f"measured {w['engine']} in this run"})
+    if t_frac is not None and t_frac > hbm_frac:
+        rec.update({"bound": "tensor", "achieved": rec["tflops"], "peak": rec["tensor_peak"], "unit": "TFLOP/s",
+                    "frac": round(t_frac, 4)})
+    else:
+        rec.update({"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(hbm_frac, 4)})
+    rec["traffic"] = traffic
+    rec["peak_kind"] = "measured in this run (burst)"
+    return rec
 
 
 class Clocks:
@@ -228,10 +364,23 @@ def run_reference(args, cfg, rank, world):
         "config": {"workload": WORKLOAD, "B_timed": 1, "T": cfg.T, "T_sampled": t_s, "H": cfg.H, "H_I": cfg.H_I,
                    "K": cfg.K, "W": cfg.W, "layers": "Full+pool(2048x8), 3x Reindex-in-pool"},
         "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "host": host_cpu()},
         "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def host_cpu():
+    """CPU model and logical core count of the host the oracle runs on."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "logical_cores": os.cpu_count()}
 
 
 def cpu_baseline(cfg, seconds_budget=30.0):
@@ -241,7 +390,8 @@ def cpu_baseline(cfg, seconds_budget=30.0):
     s = min(times)
     return {"value": round(1.0 / s, 4), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"sequence 0 of {WORKLOAD}: one decode token through all {len(cfg.layers)} layers "
-                      f"(best of {len(times)} runs, {s:.2f} s each)"}
+                      f"(best of {len(times)} runs, {s:.2f} s each; one thread: the oracle as it stands)",
+            "host": host_cpu()}
 
 
 # ---------------------------------------------------------------------- gpu --
@@ -254,6 +404,7 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
+    measured_peaks = measure_peaks(dev)
     dc = DeviceCase(cfg, device=dev)
     descs = dc.layer_descs(append_rows=True)
     ws_bytes = csa.csa_layer_workspace_size(descs)
@@ -394,18 +545,21 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     if rank != 0:
         return
-    hbm_peak, _, peak_kind = _peaks()
+    peaks = measured_peaks
+    hbm_peak = peaks["hbm_gbs"]
     value = job_tokens_per_s(cfg.B, world, ms_max)
     alg = _algorithmic_bytes(cfg)
-    # dominant kernel: the Full layer's indexer scoring over all T positions
-    name = "index_score_tc[full]" if "index_score_tc[full]" in kernels else "index_score_decode[full]"
-    nl, tot = kernels.get(name, (0, 0.0))
-    per_launch_ms = tot / nl if nl else float("nan")
-    k_bytes = cfg.B * cfg.T * 64
-    achieved = k_bytes / (per_launch_ms * 1e-3) / 1e9 if nl else None
-    src = os.path.join(ROOT, "indexer_selected_sparse_csa2_b200", "csrc",
-                       "index_tc.cu" if name.startswith("index_score_tc") else "index_decode.cu")
-    traffic = _traffic_record(src)
+    # the dominant kernel: the largest share of the step by the per-kernel events
+    work = kernel_work(cfg)
+    per_step = {k: v[1] / args.steps for k, v in kernels.items()}
+    name = max(per_step, key=per_step.get) if per_step else None
+    recs = {}
+    for k, (nl, tot) in kernels.items():
+        if k in work:
+            recs[k] = roofline_of(k, work, tot / nl if nl else None, peaks, _traffic_record(k))
+    roof = recs.get(name) or roofline_of(name, work, (kernels[name][1] / kernels[name][0]) if name else None,
+                                         peaks, None)
+    roof["share_of_step"] = round(per_step[name] / max(sum(per_step.values()), 1e-12), 4) if name else None
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -427,18 +581,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "step_hbm_gbs": round(alg / (ms_max * 1e-3) / 1e9, 1),
         "step_hbm_frac": round(alg / (ms_max * 1e-3) / 1e9 / hbm_peak, 4),
         "step_algorithmic_bytes": alg,
-        "roofline": {
-            "kernel": name,
-            "bound": "hbm",
-            "achieved": round(achieved, 1) if achieved else None,
-            "peak": hbm_peak,
-            "unit": "GB/s",
-            "frac": round(achieved / hbm_peak, 4) if achieved else None,
-            "traffic": traffic,
-            "bytes_per_launch": k_bytes,
-            "launch_ms": round(per_launch_ms, 5),
-            "peak_kind": peak_kind,
-        },
+        "roofline": roof,
+        "roofline_kernels": {k: v for k, v in recs.items() if k != name},
+        "peaks": peaks,
         "kernels": {k: {"launches": v[0], "ms_per_step": round(v[1] / args.steps, 5)} for k, v in kernels.items()},
         "kernels_note": f"from a second timed pass with an event pair around every kernel "
                         f"({round(profiled_ms, 4)} ms/step with the events)",
@@ -452,13 +597,13 @@ def run_gpu(args, cfg, rank, world, local_rank):
     if world == 1 and not args.no_prefill:
         del dc, descs, ws
         torch.cuda.empty_cache()
-        line["prefill"] = run_prefill(args, dev)
+        line["prefill"] = run_prefill(args, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds_budget=args.cpu_seconds)
     print(json.dumps(line), flush=True)
 
 
-def run_prefill(args, dev):
+def run_prefill(args, dev, peaks):
     """One prefill chunk (4096 causal queries at a 2^20-token cache): the
     step's FP4 / FP8 encodes of the new tokens, the FP8 tcgen05 indexer GEMM
     with exact per-query Top-K, and attention for every query."""
@@ -486,8 +631,7 @@ def run_prefill(args, dev):
     kern = csa.profile_collect()
     assert csa.device_status() == 0
     ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / args.prefill_steps
-    _, bf16_peak, peak_kind = _peaks()
-    fp8_peak = 2.0 * bf16_peak
+    fp8_peak = peaks["fp8_tflops"]
     P = cfg.T - cfg.n_q
     # dense indexer work: n_q x 8 heads x 64 x (keys visible to each query) x 2
     flops = sum(2.0 * cfg.H_I * cfg.d_I * (P + t + 1) for t in range(cfg.n_q))
@@ -502,7 +646,7 @@ def run_prefill(args, dev):
                        "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                        "frac": round(tflops / fp8_peak, 4) if tflops else None,
                        "flops_per_launch": flops, "launch_ms": round(main_ms, 4),
-                       "peak_kind": f"{peak_kind} bf16 x 2 (FP8 / BF16 dense ratio)"},
+                       "peak_kind": "measured fp8 in this run (own tcgen05 GEMM and cuBLAS, the larger)"},
         "attention_tflops": round(attn_flops / (kern.get("sparse_attn_tc", kern.get("sparse_attn_mma", (1, float("nan"))))[1] /
                                                 max(1, args.prefill_steps) * 1e-3) / 1e12, 1),
         "kernels": {k: {"launches": v[0], "ms_per_chunk": round(v[1] / args.prefill_steps, 4)}

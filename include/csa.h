@@ -265,6 +265,21 @@ int32_t csa_profile_snapshot(csa_kernel_time* out, int32_t max_entries);
 void csa_profile_reset(void);
 
 /* ------------------------------------------------------------------------ */
+/* Measurement kernels (no counterpart on the pages, which report no hardware
+ * figure): the roofline denominators, measured in the same run as the kernels
+ * they judge.
+ * csa_bench_copy: copy `bytes` (a multiple of 16; both pointers 16-byte
+ *   aligned) from src to dst with 128-bit loads and stores; HBM traffic is
+ *   2 * bytes.  CSA_ERR_ALIGNMENT otherwise.
+ * csa_bench_fp8_gemm: D[M][N] (fp32, row-major) = A[M][K] * B[N][K]^T with
+ *   A and B E4M3 bytes, row-major (K contiguous), on the tcgen05 tensor cores;
+ *   M a multiple of 128, N of 256, K of 128 (CSA_ERR_SHAPE otherwise);
+ *   2*M*N*K flops. */
+csa_status csa_bench_copy(const void* src, void* dst, size_t bytes, csa_stream_t stream);
+csa_status csa_bench_fp8_gemm(const uint8_t* A, const uint8_t* B, float* D, int32_t M, int32_t N, int32_t K,
+                              csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 const char* csa_status_string(int32_t status);
 /* Device-side error code recorded by a kernel whose bounded wait on an
  * mbarrier timed out (0 = none), then cleared.  Synchronises with the device

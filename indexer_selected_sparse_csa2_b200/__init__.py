@@ -99,12 +99,15 @@ _profile_enable = _sig("csa_profile_enable", _i32, [_i32])
 _profile_collect = _sig("csa_profile_collect", _i32, [ctypes.POINTER(KernelTime), _i32])
 _profile_snapshot = _sig("csa_profile_snapshot", _i32, [ctypes.POINTER(KernelTime), _i32])
 _profile_reset = _sig("csa_profile_reset", None, [])
+_bench_copy = _sig("csa_bench_copy", _i32, [_p, _p, ctypes.c_size_t, _p])
+_bench_fp8_gemm = _sig("csa_bench_fp8_gemm", _i32, [_p, _p, _p, _i32, _i32, _i32, _p])
 
 EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
-            "csa_index_noalloc_capacity", "csa_profile_snapshot", "csa_profile_reset"]
+            "csa_index_noalloc_capacity", "csa_profile_snapshot", "csa_profile_reset",
+            "csa_bench_copy", "csa_bench_fp8_gemm"]
 
 
 def profile_enable(on: bool) -> bool:
@@ -269,6 +272,22 @@ def csa_layer_step(layers, workspace=None, stream=None, device=None) -> None:
         workspace = _workspace(csa_layer_workspace_size(layers), device or "cuda")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_layer(layers, len(layers), _ptr(workspace), nbytes, _stream(stream)), "csa_layer_step")
+
+
+def csa_bench_copy(src, dst, stream=None) -> None:
+    """128-bit copy of ``src`` into ``dst`` (same byte size) by the library's
+    copy kernel (the in-run HBM peak)."""
+    nbytes = src.numel() * src.element_size()
+    assert dst.numel() * dst.element_size() >= nbytes
+    _check(_bench_copy(_ptr(src), _ptr(dst), nbytes, _stream(stream)), "csa_bench_copy")
+
+
+def csa_bench_fp8_gemm(A, B, D, stream=None) -> None:
+    """D (fp32 [M, N]) = A (E4M3 bytes [M, K]) x B (E4M3 bytes [N, K])^T on the
+    library's tcgen05 FP8 GEMM (the in-run FP8 dense peak)."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check(_bench_fp8_gemm(_ptr(A), _ptr(B), _ptr(D), M, N, K, _stream(stream)), "csa_bench_fp8_gemm")
 
 
 # ------------------------------------------------------- argument builders --

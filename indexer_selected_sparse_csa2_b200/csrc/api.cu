@@ -30,6 +30,7 @@ size_t attn_ws_bytes(const csa_attn_args* a, int share);
 int read_tc_error(bool clear);
 int read_pf_error(bool clear);
 int read_at_error(bool clear);
+int read_pk_error(bool clear);
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2, int share);
 bool attn_tc_path(const csa_attn_args* a);
 
@@ -492,7 +493,8 @@ const char* csa_status_string(int32_t s) {
 
 int32_t csa_device_status(void) {
   const int a = read_tc_error(true), b = read_pf_error(true), c = read_at_error(true);
-  return (int32_t)(a ? a : (b ? b : c));
+  const int d = read_pk_error(true);
+  return (int32_t)(a ? a : (b ? b : (c ? c : d)));
 }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

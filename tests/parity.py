@@ -51,3 +51,20 @@ def assert_close(gpu, ora, what=""):
         i = np.unravel_index(np.argmax(np.where(bad, err - bound, -np.inf)), bad.shape)
         raise AssertionError(f"{what}: {bad.sum()} elements out of tolerance; worst at {i}: "
                              f"gpu={gpu[i]!r} oracle={ora[i]!r}")
+
+
+def oracle_attend_on(case, cfg, li, t, idx_row, inputs=None):
+    """The oracle's attention of layer ``li`` for query ``t`` of ``case``'s
+    sequence over the entries of ``idx_row`` (an index row as the GPU wrote
+    it, -1 skipped) plus the layer's window rows: used where a near-tie swap
+    makes the GPU's Top-K set differ from the oracle's, so that every row's
+    attention is still checked against the oracle (on the GPU's own set)."""
+    from oracle.attention import attend
+    from oracle.quant import fp4_dequant_rows, fp8_window_dequant_rows
+    L = cfg.layers[li]
+    inp = inputs if inputs is not None else case.inputs(li)
+    sel = np.asarray(idx_row)
+    sel = sel[sel >= 0].astype(np.int64)
+    Xm = fp4_dequant_rows(case.main_entries(L.owner, sel)) if sel.size else np.zeros((0, 512))
+    Xw = fp8_window_dequant_rows(inp.window[t:t + cfg.n_win])
+    return attend(inp.q[t], np.concatenate([Xm, Xw], axis=0), cfg.softmax_scale, inp.sink)

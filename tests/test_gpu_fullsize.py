@@ -11,7 +11,7 @@ from csa_synth import get_config
 from csa_synth.configs import FULL, REINDEX, REUSE
 from oracle.case import SynthCase
 from oracle import indexer as oi
-from tests.parity import topk_diff, assert_close, check_row_format
+from tests.parity import topk_diff, assert_close, check_row_format, oracle_attend_on
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -26,9 +26,13 @@ def csa():
     return m
 
 
-def _compare_layers(cfg, dc, b, res, queries, t_index):
-    """res: oracle results for `queries`; t_index maps query rank -> device row."""
+def _compare_layers(cfg, dc, b, res, queries, case):
+    """res: oracle results of ``case`` (sequence b) for the query tokens
+    ``queries``.  Index sets by the Top-K rule; attention on every row: against
+    the oracle's result where the sets agree, else against the oracle's
+    attention over the GPU's own index set."""
     n_identical = n_rows = 0
+    inputs = {}
     for li, L in enumerate(cfg.layers):
         dl = dc.layers[li]
         r = res[li]
@@ -60,8 +64,13 @@ def _compare_layers(cfg, dc, b, res, queries, t_index):
                     topk_diff(pad(gblk), pad(oblk), lambda p: bm[p])
             if np.array_equal(g_idx, o_idx):
                 n_identical += 1
-                assert_close(dl.out[b, t].cpu().numpy(), r.out[qr], f"layer {li} b {b} t {t} out")
-                assert_close(dl.lse[b, t].cpu().numpy(), r.lse[qr], f"layer {li} b {b} t {t} lse")
+                o_out, o_lse = r.out[qr], r.lse[qr]
+            else:
+                if li not in inputs:
+                    inputs[li] = case.inputs(li)
+                o_out, o_lse = oracle_attend_on(case, cfg, li, t, g_idx, inputs[li])
+            assert_close(dl.out[b, t].cpu().numpy(), o_out, f"layer {li} b {b} t {t} out")
+            assert_close(dl.lse[b, t].cpu().numpy(), o_lse, f"layer {li} b {b} t {t} lse")
     # near-tie swaps are allowed by the Top-K rule but must stay rare
     assert n_identical >= 0.75 * n_rows, (n_identical, n_rows)
 
@@ -88,7 +97,7 @@ def _run_decode(csa, name, batches, graph=False):
     csa.csa_layer_step(descs, workspace=ws)
     torch.cuda.synchronize()
     assert csa.device_status() == 0
-    results = {}
+    results, cases = {}, {}
     for b in batches:
         case = SynthCase(cfg, b, threads=os.cpu_count() or 4, dense_latents=True)
         for o in cfg.owners:
@@ -96,7 +105,8 @@ def _run_decode(csa, name, batches, graph=False):
             assert np.array_equal(dc.keys[o][b].cpu().numpy()[rows], case.keys(o)[rows])
             assert np.array_equal(dc.kv[o][b, torch.from_numpy(rows)].cpu().numpy(), case.main_entries(o, rows))
         results[b] = case.run(keep_scores=True)
-        _compare_layers(cfg, dc, b, results[b], [0], None)
+        cases[b] = case
+        _compare_layers(cfg, dc, b, results[b], [0], cases[b])
     if graph:
         g = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream()
@@ -110,7 +120,7 @@ def _run_decode(csa, name, batches, graph=False):
         torch.cuda.synchronize()
         assert csa.device_status() == 0
         for b in batches:
-            _compare_layers(cfg, dc, b, results[b], [0], None)
+            _compare_layers(cfg, dc, b, results[b], [0], cases[b])
         del g
 
 
@@ -140,4 +150,4 @@ def test_fullsize_prefill_1m(csa):
     qs = [0, 1, 2047, 4095]
     case = SynthCase(cfg, 0, threads=os.cpu_count() or 4, dense_latents=True)
     res = case.run(queries=qs, keep_scores=True)
-    _compare_layers(cfg, dc, 0, res, qs, None)
+    _compare_layers(cfg, dc, 0, res, qs, case)

@@ -11,7 +11,7 @@ from csa_synth.configs import FULL, REINDEX, REUSE
 from oracle.case import SynthCase
 from oracle import indexer as oi
 from oracle import quant as oq
-from tests.parity import topk_diff, assert_close, check_row_format
+from tests.parity import topk_diff, assert_close, check_row_format, oracle_attend_on
 
 pytestmark = pytest.mark.gpu
 
@@ -73,12 +73,16 @@ def _check_stack(csa, cfg, append=False, sinks=False, batches=None, ws_fill=None
                     oblk = np.unique(r.pool[:r.pool_len] // cfg.pool_block_len)
                     pad = lambda a: np.concatenate([a, -np.ones(cfg.pool_blocks - a.size, np.int64)])
                     topk_diff(pad(gblk), pad(oblk), lambda p: bm[p])
-            # attention: compare where the index sets agree exactly
+            # attention on every row: the oracle's result where the index sets
+            # agree exactly, else the oracle's attention over the GPU's own set
             src_layer = li if L.mode != REUSE else L.reuse_from
             g_sel = dc.layers[src_layer].idx[b, 0].cpu().numpy()
             if np.array_equal(g_sel, r.idx[0]):
-                assert_close(dl.out[b, 0].cpu().numpy(), r.out[0], f"layer {li} out")
-                assert_close(dl.lse[b, 0].cpu().numpy(), r.lse[0], f"layer {li} lse")
+                o_out, o_lse = r.out[0], r.lse[0]
+            else:
+                o_out, o_lse = oracle_attend_on(case, cfg, li, 0, g_sel)
+            assert_close(dl.out[b, 0].cpu().numpy(), o_out, f"layer {li} out")
+            assert_close(dl.lse[b, 0].cpu().numpy(), o_lse, f"layer {li} lse")
 
 
 def test_tiny_decode(csa):
