@@ -24,7 +24,8 @@ void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_
 cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
                          int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream);
 size_t index_decode_ws_bytes(const csa_index_args* a);
-cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists);
+cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists,
+                             cudaEvent_t pool_done);
 size_t index_hist_bytes(const csa_index_args* a);
 size_t attn_ws_bytes(const csa_attn_args* a, int share);
 int read_tc_error(bool clear);
@@ -134,36 +135,38 @@ csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t works
   const size_t need = index_decode_ws_bytes(a);
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
-  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream, nullptr));
+  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream, nullptr, nullptr));
 }
 
 size_t csa_topk_workspace_size(int32_t B, int64_t n) {
   if (B < 1 || n < 1) return 0;
-  return select_workspace_bytes(B, n);
+  return ((size_t)B * kHistBins * 4 + 255) & ~(size_t)255;
 }
 
 csa_status csa_topk_scores(const float* scores, int32_t B, int64_t n, int64_t row_stride, int32_t K,
                            int32_t* idx, void* workspace, size_t workspace_bytes, csa_stream_t stream) {
   if (!scores || !idx) return CSA_ERR_INVALID_ARG;
   if (B < 1 || n < 1 || n >= ((int64_t)1 << 31) || row_stride < n || K < 1 || K > 65536) return CSA_ERR_SHAPE;
-  const size_t need = select_workspace_bytes(B, n);
+  const size_t need = csa_topk_workspace_size(B, n);
   if (need > workspace_bytes || !workspace) return CSA_ERR_WORKSPACE;
   if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
   cudaStream_t st = (cudaStream_t)stream;
-  SelectJob j{};
-  select_carve(j, B, n, workspace);
+  uint32_t* hist = static_cast<uint32_t*>(workspace);
+  cudaError_t e = launch_zero(hist, (size_t)B * kHistBins * 4, st);
+  if (e == cudaSuccess) e = launch_hist_only(scores, row_stride, n, nullptr, hist, B, st);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  CsRow j{};
   j.vals = scores;
   j.row_stride = row_stride;
-  j.n_row = nullptr;
+  j.vec = (row_stride % 4) == 0 && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+  j.n = n;
+  j.hist = hist;
   j.K = K;
   j.out = idx;
   j.out_stride = K;
   j.out_width = K;
-  j.map = nullptr;
-  j.expand = 0;
-  cudaError_t e = launch_zero(j.hist, (size_t)B * kHistBins * 4, st);
-  if (e != cudaSuccess) return CSA_ERR_CUDA;
-  return from_cuda(launch_select(&j, 1, B, true, st));
+  j.run = cs_run(n);
+  return from_cuda(launch_cluster_select(&j, 1, B, st, "topk_select"));
 }
 
 size_t csa_attn_workspace_size(const csa_attn_args* a) {
@@ -319,6 +322,7 @@ struct StackStreams {
   cudaEvent_t pro = nullptr;     // prologue (appends, histogram clearing) done
   cudaEvent_t stg = nullptr;     // decode queries staged
   cudaEvent_t idx[kMaxStackLayers] = {};
+  cudaEvent_t pool[kMaxStackLayers] = {};   // a pool-building layer's pool is written
   cudaEvent_t join[kAuxStreams] = {};   // tail of an auxiliary stream, joined into the caller's
   std::mutex mu;                        // one step enqueues on this device's streams at a time
   bool ok = false;
@@ -339,7 +343,8 @@ static StackStreams* stack_streams() {
            cudaEventCreateWithFlags(&S.start, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&S.stg, cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < kMaxStackLayers && good; ++i)
-      good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess;
+      good = cudaEventCreateWithFlags(&S.idx[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&S.pool[i], cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < kAuxStreams && good; ++i)
       good = cudaEventCreateWithFlags(&S.join[i], cudaEventDisableTiming) == cudaSuccess;
     if (!good) return nullptr;
@@ -453,11 +458,11 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       const int share = attn_share(layers, n_layers, i);
       reg_off += layer_region_bytes(L, ix, at, share);
       if (L.mode != CSA_MODE_REUSE) {
-        if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->idx[L.pool_from], 0) != cudaSuccess)
+        if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->pool[L.pool_from], 0) != cudaSuccess)
           return CSA_ERR_CUDA;
         uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
         hist_off += index_hist_bytes(&ix);
-        if (run_index_decode(&ix, region, ls, h) != cudaSuccess) return CSA_ERR_CUDA;
+        if (run_index_decode(&ix, region, ls, h, ix.pool_out ? SS->pool[i] : nullptr) != cudaSuccess) return CSA_ERR_CUDA;
       } else if (cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
         return CSA_ERR_CUDA;
       }

@@ -112,20 +112,24 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// A kernel's dynamic shared-memory limit, raised once per device:
-// cudaFuncSetAttribute applies to the current device only, so a process that
-// drives several GPUs must set it on each.  Thread-safe (a race sets it twice,
-// which is harmless).
+// A kernel attribute (set(): its dynamic shared-memory limit; set_attr(): any
+// other), set once per device: cudaFuncSetAttribute applies to the current
+// device only, so a process that drives several GPUs must set it on each.
+// Thread-safe (a race sets it twice, which is harmless).
 class SmemAttrOnce {
  public:
   template <typename... KArgs>
   cudaError_t set(void (*kernel)(KArgs...), size_t bytes) {
+    return set_attr(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  }
+  template <typename... KArgs>
+  cudaError_t set_attr(void (*kernel)(KArgs...), cudaFuncAttribute which, int value) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t)1 << dev : 0;
     if (bit && (done_.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    e = cudaFuncSetAttribute(kernel, which, value);
     if (e == cudaSuccess && bit) done_.fetch_or(bit, std::memory_order_acq_rel);
     return e;
   }

@@ -196,10 +196,10 @@ cudaError_t launch_score_decode(const ScoreParams& p, int B, cudaStream_t stream
 
 // ----------------------------------------------------------- entry point --
 struct IndexWs {
-  float* scores;
-  float* bmax;
-  SelectJob pos;
-  SelectJob blk;
+  uint32_t* hist;            // [B][4096] first-level histogram of the scores
+  uint32_t* bhist;           // [B][4096] ... of the block maxima (pool build)
+  float* scores;             // [B][n] (unless the caller takes them)
+  float* bmax;               // [B][nb] block maxima (pool build)
   size_t bytes;
 };
 
@@ -207,6 +207,10 @@ static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
                             int64_t nb, cudaStream_t stream);
+
+// Pool searches whose slots fit the fused cluster kernel score and select in
+// one launch and need no workspace.
+static bool fused_pool(const csa_index_args* a) { return a->pool && cs_pool_ok(a->pool_cap); }
 
 // Workspace layout of one decode index call.
 static IndexWs carve_index_ws(const csa_index_args* a, void* ws) {
@@ -216,16 +220,17 @@ static IndexWs carve_index_ws(const csa_index_args* a, void* ws) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   size_t off = 0;
   // both first-level histograms side by side, cleared by one launch
-  uint32_t* hists = reinterpret_cast<uint32_t*>(base);
+  w.hist = reinterpret_cast<uint32_t*>(base);
+  w.bhist = w.hist + (size_t)B * kHistBins;
   off += al256((size_t)2 * B * kHistBins * 4);
-  w.scores = reinterpret_cast<float*>(base + off); off += al256((size_t)B * n * 4);
-  off += select_carve(w.pos, B, n, base ? base + off : nullptr);
-  w.pos.hist = hists;
+  if (!fused_pool(a)) {
+    w.scores = reinterpret_cast<float*>(base + off);
+    off += al256((size_t)B * n * 4);
+  }
   if (a->pool_out) {
     const int64_t nb = (a->T + a->pool_block_len - 1) / a->pool_block_len;
-    w.bmax = reinterpret_cast<float*>(base + off); off += al256((size_t)B * nb * 4);
-    off += select_carve(w.blk, B, nb, base ? base + off : nullptr);
-    w.blk.hist = hists + (size_t)B * kHistBins;
+    w.bmax = reinterpret_cast<float*>(base + off);
+    off += al256((size_t)B * nb * 4);
   }
   w.bytes = off;
   return w;
@@ -245,81 +250,121 @@ size_t index_hist_bytes(const csa_index_args* a) {
 
 // `hists`: optional region of index_hist_bytes(a) that the caller has already
 // cleared (a layer stack clears all its layers' histograms in one launch);
-// without it the workspace's own histograms are cleared here.
-cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists) {
+// without it the workspace's own histograms are cleared here.  `pool_done`:
+// optional event recorded once the candidate pool is written (before the
+// position Top-K of a pool-building call), so that layers searching the pool
+// can start early.
+cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists,
+                             cudaEvent_t pool_done) {
   if (a->n_q > 1) return run_index_prefill(a, ws, stream);
   IndexWs w = carve_index_ws(a, ws);
   const int B = a->B;
   const int64_t n = a->pool ? (int64_t)a->pool_cap : a->T;
   cudaError_t e;
-  if (hists) {
-    w.pos.hist = hists;
-    if (a->pool_out) w.blk.hist = hists + (size_t)B * kHistBins;
-  } else {
-    // histograms start at zero (both sit at the start of the workspace)
-    e = launch_zero(w.pos.hist, (size_t)(a->pool_out ? 2 : 1) * B * kHistBins * 4, stream);
-    if (e != cudaSuccess) return e;
-  }
-  ScoreParams p{};
-  p.keys = a->keys;
-  p.key_row_stride = a->key_row_stride;
-  p.key_batch_stride = a->key_batch_stride;
-  p.q = a->q;
-  p.w = a->w;
-  p.H_I = a->H_I;
-  p.pool = a->pool;
-  p.pool_len = a->pool_len;
-  p.n = n;
-  p.chunk = score_chunk(B, n);
-  p.scores = a->scores ? a->scores : w.scores;
-  p.hist = w.pos.hist;
-  if (a->pool_out) {
-    p.bmax = w.bmax;
-    p.bhist = w.blk.hist;
-    p.nb = (a->T + a->pool_block_len - 1) / a->pool_block_len;
-    p.block_len = a->pool_block_len;
-  }
-  // full scans run on the tcgen05 scorer; pool searches gather rows and use
-  // the mma.sync scorer
-  if (a->pool) e = launch_score_decode(p, B, stream);
-  else e = launch_score_tc(a, p.scores, p.hist, p.bmax, p.bhist, p.nb, stream);
-  if (e != cudaSuccess) return e;
+  float* scores = a->scores ? a->scores : w.scores;
 
-  SelectJob jobs[2];
-  int nj = 0;
-  SelectJob& jp = w.pos;
-  jp.vals = p.scores;
-  jp.row_stride = n;
-  jp.n_row = a->pool ? a->pool_len : nullptr;
+  CsRow jp{};
+  jp.n = n;
   jp.K = a->K;
   jp.out = a->idx;
   jp.out_stride = a->K;
   jp.out_width = a->K;
-  jp.map = a->pool;
-  jp.map_stride = a->pool_cap;
-  jp.expand = 0;
-  jp.out_len = nullptr;
-  jp.limit = 0;
-  jobs[nj++] = jp;
+  jp.run = cs_run(n);
+  if (fused_pool(a)) {
+    // Reindex inside the pool: gather + score + select in one cluster launch
+    jp.row_stride = a->pool_cap;
+    jp.map = a->pool;
+    jp.map_stride = a->pool_cap;
+    CsPool pp{};
+    pp.keys = a->keys;
+    pp.key_row_stride = a->key_row_stride;
+    pp.key_batch_stride = a->key_batch_stride;
+    pp.q = a->q;
+    pp.w = a->w;
+    pp.H_I = a->H_I;
+    pp.pool_len = a->pool_len;
+    pp.scores = a->scores;
+    return launch_cluster_pool_select(jp, pp, B, stream);
+  }
+
+  if (hists) {
+    w.hist = hists;
+    w.bhist = hists + (size_t)B * kHistBins;
+  } else {
+    // histograms start at zero (both sit at the start of the workspace)
+    e = launch_zero(w.hist, (size_t)(a->pool_out ? 2 : 1) * B * kHistBins * 4, stream);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t nb = a->pool_out ? (a->T + a->pool_block_len - 1) / a->pool_block_len : 0;
+  if (a->pool) {
+    // pool rows too long for the fused kernel: gathered scoring, then the select
+    ScoreParams p{};
+    p.keys = a->keys;
+    p.key_row_stride = a->key_row_stride;
+    p.key_batch_stride = a->key_batch_stride;
+    p.q = a->q;
+    p.w = a->w;
+    p.H_I = a->H_I;
+    p.pool = a->pool;
+    p.pool_len = a->pool_len;
+    p.n = n;
+    p.chunk = score_chunk(B, n);
+    p.scores = scores;
+    p.hist = w.hist;
+    e = launch_score_decode(p, B, stream);
+  } else {
+    e = launch_score_tc(a, scores, w.hist, w.bmax, w.bhist, nb, stream);
+  }
+  if (e != cudaSuccess) return e;
+
   if (a->pool_out) {
-    SelectJob& jb = w.blk;
+    // the candidate pool first: the pool layers wait only for it
+    CsRow jb{};
     jb.vals = w.bmax;
-    jb.row_stride = p.nb;
-    jb.n_row = nullptr;
+    jb.row_stride = nb;
+    jb.vec = (nb % 4) == 0;
+    jb.n = nb;
+    jb.hist = w.bhist;
     jb.K = a->pool_blocks;
     jb.out = a->pool_out;
     jb.out_stride = (int64_t)a->pool_blocks * a->pool_block_len;
     jb.out_width = a->pool_blocks * a->pool_block_len;
-    jb.map = nullptr;
-    jb.map_stride = 0;
     jb.expand = a->pool_block_len;
     jb.out_len = a->pool_out_len;
     jb.limit = a->T;
-    jobs[nj++] = jb;
+    jb.run = cs_run(nb);
+    e = launch_cluster_select(&jb, 1, B, stream, "pool_select");
+    if (e != cudaSuccess) return e;
+    if (pool_done && cudaEventRecord(pool_done, stream) != cudaSuccess) return cudaErrorUnknown;
   }
-  // the Reindex layers' pool rows fit one CTA each
-  if (nj == 1 && select_small_ok(jobs[0])) return launch_select_small(jobs[0], B, stream);
-  return launch_select(jobs, nj, B, false, stream);
+  const int64_t pool_cap = (int64_t)a->pool_blocks * a->pool_block_len;
+  if (a->pool_out && a->pool_blocks >= a->K && cs_pool_ok(pool_cap)) {
+    // The K best positions lie in the pool once it keeps >= K blocks: take any
+    // of them, p, in block c.  Were c outside the pool, the pool's blocks
+    // would all rank above c (larger max, or the same max and a lower block),
+    // and each block's first position holding its max would rank above p
+    // (larger score, or the same score at a lower position): pool_blocks >= K
+    // positions ahead of p, so p would not be among the K best.  Selecting
+    // over the pool's positions (scores gathered by position) is therefore
+    // the same as selecting over all T, ties included.
+    jp.row_stride = pool_cap;
+    jp.n = pool_cap;
+    jp.map = a->pool_out;
+    jp.map_stride = pool_cap;
+    CsPool pp{};
+    pp.pool_len = a->pool_out_len;
+    pp.gscores = scores;
+    pp.gscore_stride = a->T;
+    return launch_cluster_pool_select(jp, pp, B, stream);
+  }
+  jp.vals = scores;
+  jp.row_stride = n;
+  jp.vec = (n % 4) == 0 && ((reinterpret_cast<uintptr_t>(scores) & 15) == 0);
+  jp.n_row = a->pool ? a->pool_len : nullptr;
+  jp.hist = w.hist;
+  jp.map = a->pool;
+  jp.map_stride = a->pool_cap;
+  return launch_cluster_select(&jp, 1, B, stream, "topk_select");
 }
 
 }  // namespace csa

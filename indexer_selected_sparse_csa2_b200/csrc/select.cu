@@ -553,6 +553,27 @@ __global__ void __launch_bounds__(kSmallThreads, 1) select_small_kernel(SelectJo
     out[jj] = -1;
 }
 
+cudaError_t launch_hist_only(const float* vals, int64_t row_stride, int64_t n, const int32_t* n_row,
+                             uint32_t* hist, int B, cudaStream_t stream) {
+  SelectJobs js;
+  SelectPlan p = plan_select(B, n);
+  SelectJob& j = js.j[0];
+  j = SelectJob{};
+  j.vals = vals;
+  j.row_stride = row_stride;
+  j.n = n;
+  j.n_row = n_row;
+  j.hist = hist;
+  j.chunk = p.chunk;
+  j.nchunks = p.nchunks;
+  js.j[1] = j;
+  dim3 g((p.nchunks + kRunsPerCta - 1) / kRunsPerCta, B, 1);
+  ProfScope ps(stream, "select_hist");
+  launch_k(select_hist_kernel, dim3(g), dim3(256), 0, stream, js);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 bool select_small_ok(const SelectJob& j) { return j.n <= kSmallCap && j.expand == 0 && j.hist != nullptr; }
 
 cudaError_t launch_select_small(const SelectJob& j, int B, cudaStream_t stream) {

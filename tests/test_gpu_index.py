@@ -143,6 +143,34 @@ def test_reindex_over_pool(csa):
         assert np.all(err <= 1e-5 * np.maximum(np.abs(S), 1e-3))
 
 
+@pytest.mark.parametrize("n_blocks,lens", [(9000, (72000, 71111)), (700, (0, 5600))])
+def test_reindex_pool_sizes(csa, n_blocks, lens):
+    """Pools longer than the fused pool kernel takes (gathered scoring, then the
+    select over the scores) and a row whose pool is empty (all -1)."""
+    B, T, K = 2, 200000, 512
+    kc, qc, w = _problem(400 + n_blocks, B, T, 8)
+    rng = np.random.default_rng(401)
+    cap = 8 * n_blocks
+    pools = []
+    for b in range(B):
+        blocks = np.sort(rng.choice(T // 8, size=(lens[b] + 7) // 8, replace=False))
+        pos = (blocks[:, None] * 8 + np.arange(8)).reshape(-1)[:lens[b]].astype(np.int32)
+        p = np.full(cap, -1, np.int32)
+        p[:pos.size] = pos
+        pools.append(p)
+    pool = np.stack(pools)
+    pool_len = np.array(lens, np.int32)
+    res = _run_index(csa, kc, qc, w, K, pool=pool, pool_len=pool_len)
+    for b in range(B):
+        n = int(pool_len[b])
+        if n == 0:
+            assert np.all(res["idx"][b] == -1)
+            continue
+        ora, S = oi.reindex_topk(qc[b, 0], w[b, 0], kc[b], pool[b], n, K)
+        full = oi.index_scores(qc[b, 0], w[b, 0], kc[b])
+        topk_diff(res["idx"][b], ora, lambda p: full[p])
+
+
 def _run_topk(csa, s, K):
     st = torch.from_numpy(s).cuda()
     idx = torch.full((s.shape[0], K), -7, dtype=torch.int32, device="cuda")
