@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   uint64_t* p_full = S.bars + 6;     // [2] P written, O^T rescaled (4 warp arrivals)
   uint64_t* o_done = S.bars + 8;     // one phase per PV
   uint64_t* drain = S.bars + 9;      // [2] all MMAs of an issuer retired (teardown; [1] = every PV, for the output)
+  uint64_t* q_full = S.bars + 11;    // staged query copied in by the bulk copies
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bt = blockIdx.y;
   const int b = bt / p.n_q, tq = bt - b * p.n_q;
@@ -153,7 +154,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     mbar_init(o_done, 1);
+    mbar_init(q_full, 1);
     fence_mbar_init();
+    if (p.q2) {
+      // the token's staged query: the tensor-memory part into the (still
+      // idle) entry-tile buffers, the shared-memory part straight to its place
+      const uint8_t* q2t = p.q2 + (size_t)(blockIdx.y) * kQ2TokenBytes;
+      mbar_arrive_expect_tx(q_full, kQ2TokenBytes);
+      for (int c = 0; c < kQ2TmemBytes; c += 32768) bulk_load(S.kv + c, q2t + c, 32768, q_full);
+      bulk_load(S.q2, q2t + kQ2TmemBytes, kQ2SmemBytes, q_full);
+    }
   }
 
   // gather role: 8 consecutive lanes take 8 different entries, so each
@@ -186,6 +196,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }                                                                                          \
   } while (0)
   const bool is_deq = warp >= 4 && warp < kAtWarpS;
+  // with the query staged by bulk copies the gather warps are free: the first
+  // tile's loads go out now, under the staging
+  if (p.q2 && is_deq && nt > 0) CSA_AT_FETCH(tile0);
 
   if (warp == kAtWarpS) tmem_alloc(S.tmem_base, kAtTmemCols);
   tc_fence_before();
@@ -200,38 +213,34 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   const float* qg = p.q + (int64_t)bt * kAtH * kD;
   if (p.q2) {
     // q staged by the stack prologue: copy rows into TMEM, the rest into shared memory
-    const uint8_t* q2t = p.q2 + (size_t)bt * kQ2TokenBytes;
-    if (warp < kAtWarpS) {
-      const int qq = warp & 3, wr = warp >> 2;
-      const int r = 32 * qq + lane;
-      const uint4* src = reinterpret_cast<const uint4*>(q2t + ((size_t)r * kQ2TmemWords + 64 * wr) * 4);
+    // warps 0-3 (one TMEM lane quarter each) move the tensor-memory part
+    // from shared memory into TMEM; the shared-memory part is already in place
+    if (warp < 4) {
+      const int r = 32 * warp + lane;
+      if (!mbar_wait_warp(q_full, 0u, kErrWaitTmaFull)) {
+        // leave the query unstaged (the error flag is set)
+      } else {
+        const uint4* row = reinterpret_cast<const uint4*>(S.kv + (size_t)r * kQ2TmemWords * 4);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 48; c0 += 8) {            // 8 chunks = 32 columns per round
+          uint32_t v[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {          // 8 loads in flight per half
-        uint4 f[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) f[k] = ld_nc_v4(src + 8 * half + k);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          uint32_t v[16];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            v[4 * k] = f[4 * u + k].x; v[4 * k + 1] = f[4 * u + k].y;
-            v[4 * k + 2] = f[4 * u + k].z; v[4 * k + 3] = f[4 * u + k].w;
+          for (int k = 0; k < 8; ++k) {
+            const uint4 f = row[(c0 + k) ^ (r & 7)];
+            v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
           }
-          tmem_st16(tbase + ((uint32_t)(32 * qq) << 16) + 64u * wr + 32u * half + 16u * u, v);
+          uint32_t (&lo)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+          uint32_t (&hi)[16] = *reinterpret_cast<uint32_t(*)[16]>(v + 16);
+          tmem_st16(tbase + ((uint32_t)(32 * warp) << 16) + 4u * c0, lo);
+          tmem_st16(tbase + ((uint32_t)(32 * warp) << 16) + 4u * c0 + 16u, hi);
         }
+        tmem_wait_st();
       }
-      tmem_wait_st();
+    } else if (is_deq) {
+      // the entry-tile buffers hold the staged query until the barrier below
+    } else {
+      mbar_wait_warp(q_full, 0u, kErrWaitTmaFull);     // S.q2 written before the MMAs read it
     }
-    const uint4* src = reinterpret_cast<const uint4*>(q2t + kQ2TmemBytes);
-    uint4* dst = reinterpret_cast<uint4*>(S.q2);
-    constexpr int kN = kQ2SmemBytes / 16;
-    constexpr int kIt = (kN + kAtThreads - 1) / kAtThreads;
-    uint4 f[kIt];
-#pragma unroll
-    for (int t = 0; t < kIt; ++t) if (tid + t * kAtThreads < kN) f[t] = ld_nc_v4(src + tid + t * kAtThreads);
-#pragma unroll
-    for (int t = 0; t < kIt; ++t) if (tid + t * kAtThreads < kN) dst[tid + t * kAtThreads] = f[t];
   } else {
   if (warp < kAtWarpS) {
     const int qq = warp & 3, wr = warp >> 2;
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     }
   } else if (is_deq) {
     // --------------------------------------------------- gather + dequantise
-    if (nt > 0) CSA_AT_FETCH(tile0);
+    if (!p.q2 && nt > 0) CSA_AT_FETCH(tile0);
     for (int i = 0; i < nt; ++i) {
       const int bi = i & 1;
       if (i >= 2 && !mbar_wait_warp(kv_free + bi, (uint32_t)((i >> 1) - 1) & 1u, kErrWaitSmemEmpty)) break;

@@ -3,7 +3,10 @@
 // h's query and row 2h+1 the lo part fp16(q - hi); inside each group of 8
 // channels the order is (0, 4, 1, 5, 2, 6, 3, 7).  Channels 0..383 are the
 // part that lives in tensor memory (row-major, 192 32-bit words per row: word
-// j = the fp16 pair (8g + (j & 3), 8g + (j & 3) + 4), g = j / 4); channels
+// j = the fp16 pair (8g + (j & 3), 8g + (j & 3) + 4), g = j / 4; the 16-byte
+// chunk of group g is stored at chunk position g ^ (r & 7) of row r, so that a
+// warp reading one chunk of 32 consecutive rows from shared memory touches
+// every bank once per 8 rows); channels
 // 384..511 the part that lives in shared memory (two K-major 128-byte-swizzled
 // blocks of 128 rows x 64 channels).  A decode step can build this once per
 // token (prologue) and every split CTA copies it instead of converting q.
@@ -53,7 +56,7 @@ CSA_DEV void encode_q2_head(const float* q_tok, int h, int lane, uint8_t* q2_tok
       const int r = 2 * h + part;
       uint8_t* dst;
       if (g < 48) {
-        dst = q2_tok + ((size_t)r * kQ2TmemWords + 4 * g) * 4;
+        dst = q2_tok + ((size_t)r * kQ2TmemWords + 4 * (g ^ (r & 7))) * 4;
       } else {
         const int kb = (g - 48) >> 3, c8 = (g - 48) & 7;
         dst = q2_tok + kQ2TmemBytes + kb * (128 * 128) + sw128_offset_h(r, 8 * c8);

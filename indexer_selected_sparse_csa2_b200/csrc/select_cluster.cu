@@ -88,41 +88,6 @@ struct CsSmem {
   uint32_t hist_red[kHistBins];                   // owner CTAs: the merged 4096-bin histogram
 };
 
-// ------------------------------------------------------ cluster primitives --
-CSA_DEV uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-CSA_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-CSA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-CSA_DEV void cluster_sync_all() {
-  cluster_arrive();
-  cluster_wait();
-}
-// Address of this CTA's shared variable `p` as seen in CTA `rank` of the cluster.
-CSA_DEV uint32_t dsmem(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
-}
-CSA_DEV void dsmem_add(uint32_t addr, uint32_t v) {
-  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-CSA_DEV void dsmem_st(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-CSA_DEV uint32_t dsmem_atom_add(uint32_t addr, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
-  return old;
-}
-CSA_DEV uint32_t dsmem_ld(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
-}
-
 // Inclusive scan over the 1024 threads; *total gets the sum.  Ends with a
 // barrier, so the scratch may be reused right away.
 CSA_DEV uint32_t cs_block_scan(uint32_t v, uint32_t* wtot, uint32_t* total) {

@@ -81,6 +81,14 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// Untiled bulk copy global -> this CTA's shared memory (no multicast):
+// addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
+CSA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
 CSA_DEV void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -170,6 +178,60 @@ CSA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
 CSA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Named barrier over `count` threads (warps of one role).
 CSA_DEV void named_bar(int id, int count) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory"); }
+
+// ------------------------------------------------------ cluster primitives --
+// Thread-block clusters and distributed shared memory: a CTA addresses a
+// peer's shared variable through mapa; barrier.cluster is a hardware barrier
+// over every thread of every CTA of the cluster (arrive and wait may be split
+// to overlap the wait with other work).  A CTA must not touch a peer's shared
+// memory before the peer has started (a first barrier) nor leave while a
+// peer may still touch its own (a last barrier after the final access).
+CSA_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+CSA_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+CSA_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+CSA_DEV void cluster_sync_all() {
+  cluster_arrive();
+  cluster_wait();
+}
+// Address of this CTA's shared variable `p` as seen in CTA `rank` of the cluster.
+CSA_DEV uint32_t dsmem(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+CSA_DEV void dsmem_add(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+CSA_DEV void dsmem_st(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+CSA_DEV uint32_t dsmem_atom_add(uint32_t addr, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+  return old;
+}
+CSA_DEV uint32_t dsmem_ld(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+CSA_DEV void dsmem_st_v2f(uint32_t addr, float2 v) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
+// No memory clobber: a caller that issues several of these back to back keeps
+// them all in flight (ordering against peers' writes comes from the cluster
+// barrier, itself a compiler memory barrier).
+CSA_DEV float4 dsmem_ld_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
 
 // ------------------------------------------------------------- descriptors --
 // Shared-memory matrix descriptor, K-major, 64-byte swizzle: rows of 64 bytes,
