@@ -265,6 +265,44 @@ int32_t csa_profile_snapshot(csa_kernel_time* out, int32_t max_entries);
 void csa_profile_reset(void);
 
 /* ------------------------------------------------------------------------ */
+/* Context-parallel decode of one long sequence.  The positions [0, T) are
+ * split into contiguous shards [t0, t1), one per rank, in rank order; each
+ * rank holds its shard's keys and main KV, the last rank also the window.
+ * The pages give no multi-GPU scheme; these kernels follow from the Top-K
+ * rule and the softmax of the calls above (Model techniques map,
+ * "Indexer-selected sparse attention" and "Multi-head latent attention"
+ * rows).  A decode step:
+ *   1. csa_index_topk on the shard (T = t1 - t0, scores requested), then
+ *      csa_cp_local_pairs: the shard's Top-K as (score, global position);
+ *   2. all-gather of the pairs over the ranks (caller: NCCL), rank-major
+ *      [R][B][K_local];
+ *   3. csa_cp_merge_topk: the global Top-K [B][K] (exact: every global
+ *      winner is among its shard's K best; ties to the lower position);
+ *   4. csa_cp_localize to this shard, csa_sparse_attn over it (sink NULL;
+ *      the window only on the last rank) -> (out_r, lse_r);
+ *   5. all-gather of (out_r, lse_r), rank-major; csa_cp_combine.
+ * All pointers are device pointers; every call is asynchronous on `stream`. */
+/* idx: [B][K] shard-local positions (-1 = none); scores: [B][score_stride]
+ * the shard's scores; writes pair_score / pair_pos [B][K] = (scores[b][p],
+ * p + t0), or (-inf, -1) for padding. */
+csa_status csa_cp_local_pairs(const int32_t* idx, const float* scores, int32_t B, int32_t K, int64_t score_stride,
+                              int64_t t0, float* pair_score, int32_t* pair_pos, csa_stream_t stream);
+/* pair_score / pair_pos: [R][B][K_local] gathered in rank order (each list
+ * ascending with trailing -1); idx: out [B][K] ascending positions, -1
+ * padded.  R <= 1024. */
+size_t csa_cp_merge_workspace_size(int32_t R, int32_t B, int32_t K_local);
+csa_status csa_cp_merge_topk(const float* pair_score, const int32_t* pair_pos, int32_t R, int32_t B,
+                             int32_t K_local, int32_t K, int32_t* idx, void* workspace, size_t workspace_bytes,
+                             csa_stream_t stream);
+/* idx_local[i] = idx[i] - t0 for idx[i] in [t0, t1), else -1 ([B][K]). */
+csa_status csa_cp_localize(const int32_t* idx, int32_t B, int32_t K, int64_t t0, int64_t t1, int32_t* idx_local,
+                           csa_stream_t stream);
+/* o_parts [R][B][H][512], lse_parts [R][B][H] (natural log; -inf for a rank
+ * with no entries); sink optional [H]; out [B][H][512], lse optional [B][H]. */
+csa_status csa_cp_combine(const float* o_parts, const float* lse_parts, int32_t R, int32_t B, int32_t H,
+                          const float* sink, float* out, float* lse, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Measurement kernels (no counterpart on the pages, which report no hardware
  * figure): the roofline denominators, measured in the same run as the kernels
  * they judge.

@@ -101,13 +101,19 @@ _profile_snapshot = _sig("csa_profile_snapshot", _i32, [ctypes.POINTER(KernelTim
 _profile_reset = _sig("csa_profile_reset", None, [])
 _bench_copy = _sig("csa_bench_copy", _i32, [_p, _p, ctypes.c_size_t, _p])
 _bench_fp8_gemm = _sig("csa_bench_fp8_gemm", _i32, [_p, _p, _p, _i32, _i32, _i32, _p])
+_cp_pairs = _sig("csa_cp_local_pairs", _i32, [_p, _p, _i32, _i32, _i64, _i64, _p, _p, _p])
+_cp_merge_ws = _sig("csa_cp_merge_workspace_size", ctypes.c_size_t, [_i32, _i32, _i32])
+_cp_merge = _sig("csa_cp_merge_topk", _i32, [_p, _p, _i32, _i32, _i32, _i32, _p, _p, ctypes.c_size_t, _p])
+_cp_localize = _sig("csa_cp_localize", _i32, [_p, _i32, _i32, _i64, _i64, _p, _p])
+_cp_combine = _sig("csa_cp_combine", _i32, [_p, _p, _i32, _i32, _i32, _p, _p, _p, _p])
 
 EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
             "csa_index_noalloc_capacity", "csa_profile_snapshot", "csa_profile_reset",
-            "csa_bench_copy", "csa_bench_fp8_gemm"]
+            "csa_bench_copy", "csa_bench_fp8_gemm", "csa_cp_local_pairs", "csa_cp_merge_workspace_size",
+            "csa_cp_merge_topk", "csa_cp_localize", "csa_cp_combine"]
 
 
 def profile_enable(on: bool) -> bool:
@@ -288,6 +294,35 @@ def csa_bench_fp8_gemm(A, B, D, stream=None) -> None:
     M, K = A.shape
     N = B.shape[0]
     _check(_bench_fp8_gemm(_ptr(A), _ptr(B), _ptr(D), M, N, K, _stream(stream)), "csa_bench_fp8_gemm")
+
+
+def csa_cp_local_pairs(idx, scores, t0: int, pair_score, pair_pos, stream=None) -> None:
+    """Shard-local Top-K (idx [B, K] or [B, 1, K]) -> (score, global position) pairs."""
+    B, K = idx.shape[0], idx.shape[-1]
+    _check(_cp_pairs(_ptr(idx), _ptr(scores), B, K, scores.stride(0), t0, _ptr(pair_score), _ptr(pair_pos),
+                     _stream(stream)), "csa_cp_local_pairs")
+
+
+def csa_cp_merge_topk(pair_score, pair_pos, K: int, idx, workspace=None, stream=None) -> None:
+    """Gathered pairs [R, B, K_local] (rank order) -> global Top-K idx [B, K]."""
+    R, B, Kl = pair_score.shape
+    if workspace is None:
+        workspace = _workspace(int(_cp_merge_ws(R, B, Kl)), pair_score.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_cp_merge(_ptr(pair_score), _ptr(pair_pos), R, B, Kl, K, _ptr(idx), _ptr(workspace), nbytes,
+                     _stream(stream)), "csa_cp_merge_topk")
+
+
+def csa_cp_localize(idx, t0: int, t1: int, idx_local, stream=None) -> None:
+    B, K = idx.shape[0], idx.shape[-1]
+    _check(_cp_localize(_ptr(idx), B, K, t0, t1, _ptr(idx_local), _stream(stream)), "csa_cp_localize")
+
+
+def csa_cp_combine(o_parts, lse_parts, out, lse=None, sink=None, stream=None) -> None:
+    """o_parts [R, B, H, 512], lse_parts [R, B, H] -> out [B, H, 512], lse [B, H]."""
+    R, B, H = lse_parts.shape
+    _check(_cp_combine(_ptr(o_parts), _ptr(lse_parts), R, B, H, _ptr(sink), _ptr(out), _ptr(lse),
+                       _stream(stream)), "csa_cp_combine")
 
 
 # ------------------------------------------------------- argument builders --
