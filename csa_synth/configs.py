@@ -22,7 +22,7 @@ import math
 from dataclasses import dataclass, field
 from typing import List, Optional
 
-FULL, REINDEX, REUSE = 0, 1, 2
+FULL, REINDEX, REUSE, SWA = 0, 1, 2, 3
 
 
 @dataclass(frozen=True)
@@ -32,6 +32,7 @@ class LayerSpec:
     reuse_from: int = -1      # REUSE: layer whose Top-K indices are reused
     build_pool: bool = False  # FULL: also build the hierarchical candidate pool
     pool_from: int = -1       # REINDEX: score only the pool built by this layer
+    m: int = 1                # tokens per cache entry of the caches this layer owns (compressor ratio)
 
 
 @dataclass(frozen=True)
@@ -73,10 +74,35 @@ class Config:
 
     @property
     def owners(self) -> List[int]:
-        return sorted({l.owner for l in self.layers})
+        """Layers whose main KV and indexer keys the stack reads (SWA layers read none)."""
+        return sorted({l.owner for l in self.layers if l.mode != SWA})
+
+    def ratio(self, owner: int) -> int:
+        """Tokens per cache entry of an owner layer's main KV and indexer keys."""
+        return self.layers[owner].m
+
+    def entries(self, owner: int) -> int:
+        """Completed cache entries of an owner layer (T tokens; a tail group waits)."""
+        return self.T // self.ratio(owner)
 
     def replace(self, **kw) -> "Config":
         return dataclasses.replace(self, **kw)
+
+
+def _ced_layers():
+    L = [LayerSpec(SWA, 0), LayerSpec(SWA, 1)]
+    for g in range(3):                                   # encoder groups, owners 2, 8, 14
+        o = 2 + 6 * g
+        L.append(LayerSpec(FULL, o, m=2))
+        L += [LayerSpec(REUSE, o, reuse_from=o) for _ in range(5)]
+    d = 20                                               # decoder owner
+    L.append(LayerSpec(FULL, d, build_pool=True))
+    L += [LayerSpec(REUSE, d, reuse_from=d) for _ in range(3)]
+    for g in range(4):
+        r = 24 + 4 * g
+        L.append(LayerSpec(REINDEX, d, pool_from=d))
+        L += [LayerSpec(REUSE, d, reuse_from=r) for _ in range(3)]
+    return L
 
 
 CONFIGS = {
@@ -99,6 +125,11 @@ CONFIGS = {
     # of 68 B, top-512): the oracle side of the next row of the scope table
     "decode_mx": Config(name="decode_mx", B=8, T=65536, H=64, H_I=32, K=512, seed=5, d_I=128,
                         key_format="mxfp4"),
+    # the pages' 40-layer causal encoder-decoder stack: 2 SWA layers, the
+    # encoder's 3 x [1 Full, 5 Reuse] over caches of one entry per 2 tokens,
+    # the decoder's [1 Full (pool), 3 Reuse] then 4 x [1 Reindex in the pool,
+    # 3 Reuse] over the decoder's own per-token caches
+    "ced_40": Config(name="ced_40", B=4, T=1 << 17, H=64, H_I=8, K=2048, seed=6, layers=_ced_layers()),
     # a quarter-size prefill chunk (profiling captures that must stay small)
     "prefill_256k": Config(name="prefill_256k", B=1, T=1 << 18, H=64, H_I=8, K=2048, seed=4,
                            n_q=1024, bf16_latents=True),

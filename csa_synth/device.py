@@ -14,7 +14,7 @@ from typing import Dict, List, Optional
 import numpy as np
 
 from . import workload as wl
-from .configs import Config, FULL, REINDEX, REUSE
+from .configs import Config, FULL, REINDEX, REUSE, SWA
 
 UPLOAD_ROWS = 1 << 16
 
@@ -54,15 +54,23 @@ class DeviceCase:
         self.keys: Dict[int, object] = {}
         self.kv: Dict[int, object] = {}
         for o in cfg.owners:
-            keys = torch.empty((B, T, cfg.d_I), dtype=torch.uint8, device=device)
-            kv = torch.empty((B, T, csa.FP4_ENTRY_BYTES), dtype=torch.uint8, device=device)
+            E, m = cfg.entries(o), cfg.ratio(o)
+            keys = torch.empty((B, E, cfg.d_I), dtype=torch.uint8, device=device)
+            kv = torch.empty((B, E, csa.FP4_ENTRY_BYTES), dtype=torch.uint8, device=device)
             for b in range(B):
-                for t0 in range(0, T, UPLOAD_ROWS):
-                    n = min(UPLOAD_ROWS, T - t0)
-                    kx = torch.from_numpy(wl.index_key(cfg, o, b, t0, n, threads=threads)).to(device)
-                    csa.csa_quant_kv(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, t0:t0 + n])
-                    mx = self._latent_tensor(wl.main_latent(cfg, o, b, t0, n, threads=threads))
-                    csa.csa_quant_kv(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, t0:t0 + n])
+                for e0 in range(0, E, UPLOAD_ROWS):
+                    n = min(UPLOAD_ROWS, E - e0)
+                    kx = torch.from_numpy(wl.index_key(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
+                    mx = self._latent_tensor(wl.main_latent(cfg, o, b, e0 * m, n * m, threads=threads))
+                    if m == 1:
+                        csa.csa_quant_kv(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, e0:e0 + n])
+                        csa.csa_quant_kv(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
+                    else:
+                        # the compressor pools each group of m token rows into one entry
+                        kg = torch.from_numpy(wl.index_gate(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
+                        mg = torch.from_numpy(wl.main_gate(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
+                        csa.csa_compress_kv(kx, kg, m, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, e0:e0 + n])
+                        csa.csa_compress_kv(mx, mg, m, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
             self.keys[o] = keys
             self.kv[o] = kv
         self.layers: List[DeviceLayer] = []
@@ -89,8 +97,8 @@ class DeviceCase:
                 dl.pool = torch.full((B, cfg.pool_blocks * cfg.pool_block_len), -7, dtype=torch.int32,
                                      device=device)
                 dl.pool_len = torch.zeros(B, dtype=torch.int32, device=device)
-            if keep_scores and L.mode != REUSE:
-                n = cfg.T
+            if keep_scores and L.mode in (FULL, REINDEX):
+                n = cfg.entries(L.owner)
                 if L.mode == REINDEX and L.pool_from >= 0:
                     n = cfg.pool_blocks * cfg.pool_block_len
                 dl.scores = torch.zeros((B, n), dtype=torch.float32, device=device)
@@ -128,7 +136,9 @@ class DeviceCase:
                     raise ValueError("prefill appends are built for one sequence")
                 jobs = []
                 t_new = cfg.T - n_new
-                if o == li:
+                if o == li and L.mode != SWA and cfg.ratio(o) == 1:
+                    # (an owner with m > 1 gains an entry only when a group of m
+                    # tokens completes; its caches are built whole above)
                     if n_new == 1:
                         mx = torch.stack([self._latent_tensor(wl.main_latent(cfg, o, b, cfg.T - 1, 1))[0]
                                           for b in range(cfg.B)])
@@ -156,14 +166,14 @@ class DeviceCase:
                 self._append_src.append(wx)
                 for k, j in enumerate(jobs):
                     d.append[k] = j
-            if L.mode != REUSE:
+            if L.mode in (FULL, REINDEX):
                 d.index = csa.index_args(
-                    keys=self.keys[o], q=dl.qI, w=dl.w, K=cfg.K, idx=dl.idx, T=cfg.T, n_q=cfg.n_q,
+                    keys=self.keys[o], q=dl.qI, w=dl.w, K=cfg.K, idx=dl.idx, T=cfg.entries(o), n_q=cfg.n_q,
                     pool_out=dl.pool, pool_out_len=dl.pool_len, pool_blocks=cfg.pool_blocks,
                     pool_block_len=cfg.pool_block_len, scores=dl.scores)
-            d.attn = csa.attn_args(q=dl.q, kv=self.kv[o], idx=None, win=dl.win, n_win=cfg.n_win,
-                                   softmax_scale=cfg.softmax_scale, out=dl.out, lse=dl.lse, sink=dl.sink,
-                                   K=0)
+            d.attn = csa.attn_args(q=dl.q, kv=self.kv[o] if L.mode != SWA else None, idx=None, win=dl.win,
+                                   n_win=cfg.n_win, softmax_scale=cfg.softmax_scale, out=dl.out, lse=dl.lse,
+                                   sink=dl.sink, K=0)
             d._keep = (getattr(d, "_keep", None), self.keys, self.kv, dl)
             descs.append(d)
         return csa.make_layer_array(descs)

@@ -29,6 +29,8 @@ class TensorId(enum.IntEnum):
     PLANT = 8           # planted-position offsets
     SINK = 9            # optional per-head sink logits
     SCORES = 10         # synthetic score rows for selection tests
+    MAIN_GATE = 11      # compressor gate logits of main-KV token rows, [B * T, 512] (m > 1 owners)
+    INDEX_GATE = 12     # compressor gate logits of indexer-key token rows, [B * T, 64]
 
 
 def tid(base: TensorId, layer: int = 0) -> int:

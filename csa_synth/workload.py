@@ -46,6 +46,22 @@ def main_latent_at(cfg: Config, owner: int, b: int, positions: np.ndarray) -> np
     return _shape_latents(cfg, x)
 
 
+def main_gate(cfg: Config, owner: int, b: int, t0: int, n: int, threads: int = 1) -> np.ndarray:
+    """fp32 [n, D] compressor gate logits of token rows [t0, t0+n) (owners with m > 1), N(0, 2^2)."""
+    return normal_rows(cfg.seed, tid(TensorId.MAIN_GATE, owner), b * cfg.T + t0, n, cfg.D, threads) * np.float32(2)
+
+
+def main_gate_at(cfg: Config, owner: int, b: int, positions: np.ndarray) -> np.ndarray:
+    """fp32 [len(positions), D] gate logits at scattered token rows."""
+    rows = b * cfg.T + np.asarray(positions, dtype=np.int64)
+    return gather_normal_rows(cfg.seed, tid(TensorId.MAIN_GATE, owner), rows, cfg.D) * np.float32(2)
+
+
+def index_gate(cfg: Config, owner: int, b: int, t0: int, n: int, threads: int = 1) -> np.ndarray:
+    """fp32 [n, d_I] compressor gate logits of indexer-key token rows, N(0, 2^2)."""
+    return normal_rows(cfg.seed, tid(TensorId.INDEX_GATE, owner), b * cfg.T + t0, n, cfg.d_I, threads) * np.float32(2)
+
+
 def window_latent(cfg: Config, layer: int, b: int) -> np.ndarray:
     """fp32 [win_rows, D] sliding-window latents of one layer and sequence."""
     R = cfg.win_rows

@@ -73,7 +73,9 @@ typedef enum {
   CSA_FMT_FP8_E4M3_PLAIN = 2
 } csa_kv_format;
 
-typedef enum { CSA_MODE_FULL = 0, CSA_MODE_REINDEX = 1, CSA_MODE_REUSE = 2 } csa_mode;
+/* SWA: a sliding-window layer (the stack's first layers): attention over the
+ * layer's window alone, no indexer, no selected entries. */
+typedef enum { CSA_MODE_FULL = 0, CSA_MODE_REINDEX = 1, CSA_MODE_REUSE = 2, CSA_MODE_SWA = 3 } csa_mode;
 
 /* ------------------------------------------------------------------------ */
 /* (a) Encode rows.
@@ -89,6 +91,22 @@ typedef enum { CSA_MODE_FULL = 0, CSA_MODE_REINDEX = 1, CSA_MODE_REUSE = 2 } csa
 csa_status csa_quant_kv(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim,
                         int64_t src_row_stride, int32_t fmt, void* dst,
                         int64_t dst_row_stride, csa_stream_t stream);
+
+/* The m-token compressor of the encoder's CSA2 layers (DeepSeek-V4.1-Flash
+ * architecture database, cache groups: the encoder's main KV and indexer K
+ * hold one shared K=V entry per 2 tokens, pooled with a gate in fp32; the
+ * ratio-1 compressor is plain).  Group n pools token rows n*m .. n*m+m-1:
+ * per channel, w_i = exp(g_i - max_j g_j) and entry = sum_i w_i x_i /
+ * sum_i w_i (fp32, exp and a correctly rounded division), then the entry is
+ * encoded as fmt (CSA_FMT_FP4_E2M1_E4M3X16 with dim 512, or
+ * CSA_FMT_FP8_E4M3_PLAIN with dim a multiple of 16).
+ *   src  : fp32 / bf16 token rows, row r at src + r * src_row_stride elements
+ *   gate : fp32 gate logits, row r at gate + r * gate_row_stride (NULL when m == 1)
+ *   dst  : entry n at dst + n * dst_row_stride bytes; 1 <= m <= 16.
+ * Entries of an incomplete tail group are the caller's to withhold. */
+csa_status csa_compress_kv(const void* src, int32_t src_dtype, const float* gate, int64_t n_groups, int32_t m,
+                           int32_t dim, int64_t src_row_stride, int64_t gate_row_stride, int32_t fmt, void* dst,
+                           int64_t dst_row_stride, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* (b) Lightning-indexer scores + Top-K (optionally building or searching the
@@ -189,8 +207,18 @@ typedef struct {
   int32_t n_win;             /* window entries per query, 0..1024 */
   float softmax_scale;
   const float* sink;         /* optional fp32 [H] sink logits */
-  float* out;                /* fp32 [B][n_q][H][D] */
+  float* out;                /* fp32 [B][n_q][H][D] (bf16 with out_bf16) */
   float* lse;                /* optional fp32 [B][n_q][H] (natural log) */
+  /* Partial RoPE around the attention (DeepSeek-V4.1-Flash architecture
+   * database: "partial RoPE (last 64 dims of Q and KV; inverse rotation on
+   * attention output)"; Model techniques map: fused RoPE-attention-RoPE-cast
+   * kernel).  Optional fp32 [B][n_q][32][2]: (cos, sin) of the 32 angles of
+   * query t's position.  When given, channels (448 + 2i, 449 + 2i) of q are
+   * rotated by angle i (x + iy times e^{i angle}) before the logits and the
+   * same channels of out are rotated back (angle negated); the cached
+   * entries are taken as already rotated.  NULL = no rotation. */
+  const float* rope_cs;
+  int32_t out_bf16;          /* 1: out is bf16 [B][n_q][H][D], round to nearest even */
 } csa_attn_args;
 
 size_t csa_attn_workspace_size(const csa_attn_args* a);
@@ -206,6 +234,7 @@ csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t works
  *             pool_cap are taken from layer pool_from's pool_out.
  *   REUSE   : no scoring; attention with attn.idx = the idx of layer
  *             reuse_from (attn.K likewise).
+ *   SWA     : no scoring; attention over the window alone (attn.K = 0).
  * `append[i]` with src != NULL encodes new rows (e.g. this step's token)
  * into the caches before any layer's scoring (all appends of the stack run
  * first, in one launch).

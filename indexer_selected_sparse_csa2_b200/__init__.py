@@ -33,7 +33,7 @@ CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_SHAPE, CSA_ERR_ALIGNMENT, CSA_ERR_UNSUPPORT
     CSA_ERR_WORKSPACE, CSA_ERR_CUDA = range(7)
 CSA_SRC_F32, CSA_SRC_BF16 = 0, 1
 CSA_FMT_FP4_E2M1_E4M3X16, CSA_FMT_FP8_E4M3_UE8M0X32, CSA_FMT_FP8_E4M3_PLAIN = 0, 1, 2
-CSA_MODE_FULL, CSA_MODE_REINDEX, CSA_MODE_REUSE = 0, 1, 2
+CSA_MODE_FULL, CSA_MODE_REINDEX, CSA_MODE_REUSE, CSA_MODE_SWA = 0, 1, 2, 3
 FP4_ENTRY_BYTES, FP8_ENTRY_BYTES = 288, 528
 
 _p = ctypes.c_void_p
@@ -56,7 +56,8 @@ class AttnArgs(ctypes.Structure):
                 ("q", _p), ("kv", _p), ("kv_row_stride", _i64), ("kv_batch_stride", _i64),
                 ("idx", _p), ("K", _i32),
                 ("win", _p), ("win_row_stride", _i64), ("win_batch_stride", _i64), ("n_win", _i32),
-                ("softmax_scale", _f32), ("sink", _p), ("out", _p), ("lse", _p)]
+                ("softmax_scale", _f32), ("sink", _p), ("out", _p), ("lse", _p),
+                ("rope_cs", _p), ("out_bf16", _i32)]
 
 
 class QuantJob(ctypes.Structure):
@@ -81,6 +82,7 @@ def _sig(name, res, args):
 
 
 _quant = _sig("csa_quant_kv", _i32, [_p, _i32, _i64, _i32, _i64, _i32, _p, _i64, _p])
+_compress = _sig("csa_compress_kv", _i32, [_p, _i32, _p, _i64, _i32, _i32, _i64, _i64, _i32, _p, _i64, _p])
 _index_ws = _sig("csa_index_workspace_size", ctypes.c_size_t, [ctypes.POINTER(IndexArgs)])
 _index = _sig("csa_index_topk", _i32, [ctypes.POINTER(IndexArgs), _p, ctypes.c_size_t, _p])
 _index_noalloc = _sig("csa_index_topk_noalloc", _i32, [ctypes.POINTER(IndexArgs), _p])
@@ -107,7 +109,7 @@ _cp_merge = _sig("csa_cp_merge_topk", _i32, [_p, _p, _i32, _i32, _i32, _i32, _p,
 _cp_localize = _sig("csa_cp_localize", _i32, [_p, _i32, _i32, _i64, _i64, _p, _p])
 _cp_combine = _sig("csa_cp_combine", _i32, [_p, _p, _i32, _i32, _i32, _p, _p, _p, _p])
 
-EXPORTED = ["csa_quant_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
+EXPORTED = ["csa_quant_kv", "csa_compress_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
@@ -206,6 +208,20 @@ def csa_quant_kv(src, fmt: int, dst, n_rows: Optional[int] = None, dim: Optional
     dst_row_stride = dst.stride(0) * dst.element_size() if dst_row_stride is None else dst_row_stride
     _check(_quant(_ptr(src), dtype, n_rows, dim, src_row_stride, fmt, _ptr(dst), dst_row_stride,
                   _stream(stream)), "csa_quant_kv")
+
+
+def csa_compress_kv(src, gate, m: int, fmt: int, dst, dst_row_stride: Optional[int] = None, stream=None) -> None:
+    """Pool groups of m token rows of ``src`` (fp32 / bf16 [n_groups * m, dim])
+    with the fp32 gate logits ``gate`` ([n_groups * m, dim], None when m == 1)
+    and encode each pooled entry into ``dst`` (uint8 rows)."""
+    torch = _torch()
+    dtype = CSA_SRC_BF16 if src.dtype == torch.bfloat16 else CSA_SRC_F32
+    n_groups = src.shape[0] // m
+    dim = src.shape[-1]
+    dst_row_stride = dst.stride(0) * dst.element_size() if dst_row_stride is None else dst_row_stride
+    _check(_compress(_ptr(src), dtype, _ptr(gate), n_groups, m, dim, src.stride(0),
+                     0 if gate is None else gate.stride(0), fmt, _ptr(dst), dst_row_stride, _stream(stream)),
+           "csa_compress_kv")
 
 
 def csa_index_workspace_size(args: IndexArgs) -> int:
@@ -351,13 +367,16 @@ def index_args(*, keys, q, w, K: int, idx, T: Optional[int] = None, n_q: int = 1
 
 
 def attn_args(*, q, kv, idx, win, n_win: int, softmax_scale: float, out, lse=None, sink=None,
-              K: Optional[int] = None) -> AttnArgs:
+              K: Optional[int] = None, rope_cs=None) -> AttnArgs:
     """AttnArgs from torch tensors: q fp32 [B, n_q, H, 512], kv uint8 [B, T, 288],
-    idx int32 [B, n_q, K], win uint8 [B, rows, 528], out fp32 [B, n_q, H, 512]."""
+    idx int32 [B, n_q, K], win uint8 [B, rows, 528], out fp32 or bf16
+    [B, n_q, H, 512]; rope_cs optional fp32 [B, n_q, 32, 2] (cos, sin) of each
+    query position's angles (partial RoPE on q, inverse rotation on out)."""
     a = AttnArgs()
     a.B, a.n_q, a.H, a.D = q.shape
     a.q = _ptr(q)
-    a.kv, a.kv_row_stride, a.kv_batch_stride = _ptr(kv), kv.stride(1), kv.stride(0)
+    if kv is not None:
+        a.kv, a.kv_row_stride, a.kv_batch_stride = _ptr(kv), kv.stride(1), kv.stride(0)
     a.idx = _ptr(idx)
     a.K = idx.shape[-1] if (K is None and idx is not None) else (K or 0)
     if win is not None:
@@ -365,7 +384,9 @@ def attn_args(*, q, kv, idx, win, n_win: int, softmax_scale: float, out, lse=Non
     a.n_win = n_win
     a.softmax_scale = softmax_scale
     a.sink, a.out, a.lse = _ptr(sink), _ptr(out), _ptr(lse)
-    a._keep = (q, kv, idx, win, out, lse, sink)
+    a.rope_cs = _ptr(rope_cs)
+    a.out_bf16 = 1 if str(out.dtype) == "torch.bfloat16" else 0
+    a._keep = (q, kv, idx, win, out, lse, sink, rope_cs)
     return a
 
 

@@ -23,6 +23,9 @@ void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_
 
 cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
                          int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream);
+cudaError_t launch_compress(const void* src, int src_dtype, const float* gate, int64_t n_groups, int m, int dim,
+                            int64_t src_row_stride, int64_t gate_row_stride, int fmt, void* dst,
+                            int64_t dst_row_stride, cudaStream_t stream);
 size_t index_decode_ws_bytes(const csa_index_args* a);
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists,
                              cudaEvent_t pool_done);
@@ -102,7 +105,8 @@ static csa_status check_attn(const csa_attn_args* a) {
   if (a->n_win > 0 && (a->win_row_stride < kFp8Bytes || !al16(a->win) || !al16i(a->win_row_stride) ||
                        !al16i(a->win_batch_stride)))
     return a->win_row_stride < kFp8Bytes ? CSA_ERR_SHAPE : CSA_ERR_ALIGNMENT;
-  if (!al16(a->q) || !al16(a->out)) return CSA_ERR_ALIGNMENT;
+  if (!al16(a->q) || !al16(a->out) || !al16(a->rope_cs)) return CSA_ERR_ALIGNMENT;
+  if (a->out_bf16 != 0 && a->out_bf16 != 1) return CSA_ERR_INVALID_ARG;
   return CSA_OK;
 }
 
@@ -121,6 +125,25 @@ csa_status csa_quant_kv(const void* src, int32_t src_dtype, int64_t n_rows, int3
   if (s != CSA_OK || n_rows == 0) return s;
   return from_cuda(launch_quant(src, src_dtype, n_rows, dim, src_row_stride, fmt, dst, dst_row_stride,
                                 (cudaStream_t)stream));
+}
+
+csa_status csa_compress_kv(const void* src, int32_t src_dtype, const float* gate, int64_t n_groups, int32_t m,
+                           int32_t dim, int64_t src_row_stride, int64_t gate_row_stride, int32_t fmt, void* dst,
+                           int64_t dst_row_stride, csa_stream_t stream) {
+  if (src_dtype != CSA_SRC_F32 && src_dtype != CSA_SRC_BF16) return CSA_ERR_INVALID_ARG;
+  if (fmt != CSA_FMT_FP4_E2M1_E4M3X16 && fmt != CSA_FMT_FP8_E4M3_PLAIN) return CSA_ERR_INVALID_ARG;
+  if (n_groups < 0 || m < 1 || m > 16) return CSA_ERR_SHAPE;
+  if (n_groups == 0) return CSA_OK;
+  if (!src || !dst || (m > 1 && !gate)) return CSA_ERR_INVALID_ARG;
+  if (fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? dim != kD : (dim <= 0 || dim % 16)) return CSA_ERR_SHAPE;
+  if (src_row_stride < dim || (m > 1 && gate_row_stride < dim)) return CSA_ERR_SHAPE;
+  const int64_t esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  const int64_t row_bytes = fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? kFp4Bytes : dim;
+  if (n_groups > 1 && dst_row_stride < row_bytes) return CSA_ERR_SHAPE;
+  if (!al16(src) || !al16i(src_row_stride * esz) || !al16(dst) || !al16i(dst_row_stride)) return CSA_ERR_ALIGNMENT;
+  if (m > 1 && (!al16(gate) || !al16i(gate_row_stride * 4))) return CSA_ERR_ALIGNMENT;
+  return from_cuda(launch_compress(src, src_dtype, gate, n_groups, m, dim, src_row_stride, gate_row_stride, fmt, dst,
+                                   dst_row_stride, (cudaStream_t)stream));
 }
 
 size_t csa_index_workspace_size(const csa_index_args* a) {
@@ -184,10 +207,18 @@ csa_status csa_sparse_attn(const csa_attn_args* a, void* workspace, size_t works
   return from_cuda(run_sparse_attn(a, workspace, (cudaStream_t)stream, nullptr, 1));
 }
 
+// Layers that run the indexer (Full, Reindex); Reuse and SWA layers do not.
+static bool indexes(int32_t mode) { return mode == CSA_MODE_FULL || mode == CSA_MODE_REINDEX; }
+
 // Resolve one layer of a stack into concrete index / attention arguments.
 static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_args* ix, csa_attn_args* at) {
   const csa_layer_desc& d = L[i];
   *at = d.attn;
+  if (d.mode == CSA_MODE_SWA) {
+    at->idx = nullptr;
+    at->K = 0;
+    return CSA_OK;
+  }
   if (d.mode == CSA_MODE_REUSE) {
     if (d.reuse_from < 0 || d.reuse_from >= i) return CSA_ERR_INVALID_ARG;
     int32_t src = d.reuse_from;
@@ -195,6 +226,7 @@ static csa_status resolve_layer(const csa_layer_desc* L, int32_t i, csa_index_ar
       if (L[src].reuse_from < 0 || L[src].reuse_from >= src) return CSA_ERR_INVALID_ARG;
       src = L[src].reuse_from;
     }
+    if (L[src].mode == CSA_MODE_SWA) return CSA_ERR_INVALID_ARG;   // a window layer has no indices
     if (L[src].index.n_q != at->n_q || L[src].index.B != at->B) return CSA_ERR_SHAPE;
     at->idx = L[src].index.idx;
     at->K = L[src].index.K;
@@ -267,7 +299,7 @@ static int attn_share(const csa_layer_desc* L, int32_t n_layers, int32_t i) {
 static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& ix, const csa_attn_args& at,
                                  int share) {
   size_t r = attn_ws_bytes(&at, share);
-  if (L.mode != CSA_MODE_REUSE) r = std::max(r, index_decode_ws_bytes(&ix));
+  if (indexes(L.mode)) r = std::max(r, index_decode_ws_bytes(&ix));
   return al256(r);
 }
 
@@ -284,7 +316,7 @@ static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, Stack
       s = check_quant(q.src, q.src_dtype, q.n_rows, q.dim, q.src_row_stride, q.fmt, q.dst, q.dst_row_stride);
       if (s != CSA_OK) return s;
     }
-    if (layers[i].mode != CSA_MODE_REUSE) {
+    if (indexes(layers[i].mode)) {
       s = check_index(&ix);
       if (s != CSA_OK) return s;
       w.hists += index_hist_bytes(&ix);
@@ -388,7 +420,8 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
     qb.zero_n16 = (int64_t)(w.hists / 16);
     cudaStream_t sst = SS->aux[kAuxStreams - 1];
     auto add_job = [&](QuantBatch& q, cudaStream_t qs_stream, const void* src, int64_t n_rows,
-                       int64_t src_stride_bytes, void* dst, int64_t dst_stride, int fmt, int bf16, int dim) -> bool {
+                       int64_t src_stride_bytes, void* dst, int64_t dst_stride, int fmt, int bf16, int dim,
+                       const float* aux) -> bool {
       if (q.njobs == kMaxBatchJobs) {
         if (launch_quant_batch(q, qs_stream) != cudaSuccess) return false;
         q.njobs = 0;
@@ -404,6 +437,7 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       J.fmt = fmt;
       J.bf16 = bf16;
       J.dim = dim;
+      J.aux = aux;
       J.unit0 = q.units;
       q.units += quant_batch_units(fmt, n_rows, dim);
       return true;
@@ -421,14 +455,15 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
         if (!q.src || q.n_rows == 0) continue;
         const int esz = q.src_dtype == CSA_SRC_BF16 ? 2 : 4;
         if (!add_job(qb, st, q.src, q.n_rows, q.src_row_stride * esz, q.dst, q.dst_row_stride, q.fmt,
-                     q.src_dtype == CSA_SRC_BF16, q.dim))
+                     q.src_dtype == CSA_SRC_BF16, q.dim, nullptr))
           return CSA_ERR_CUDA;
       }
       csa_index_args ix{};
       csa_attn_args at{};
       resolve_layer(layers, i, &ix, &at);
       if (layer_q2_bytes(at)) {
-        if (!add_job(qs, sst, at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512))
+        if (!add_job(qs, sst, at.q, (int64_t)at.B * 64, 0, q2_base + q2_off, kQ2TokenBytes, kFmtStageQ2, 0, 512,
+                     at.rope_cs))
           return CSA_ERR_CUDA;
         q2_off += layer_q2_bytes(at);
       }
@@ -457,13 +492,14 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       uint8_t* region = base + reg_off;
       const int share = attn_share(layers, n_layers, i);
       reg_off += layer_region_bytes(L, ix, at, share);
-      if (L.mode != CSA_MODE_REUSE) {
+      if (indexes(L.mode)) {
         if (L.mode == CSA_MODE_REINDEX && L.pool_from >= 0 && cudaStreamWaitEvent(ls, SS->pool[L.pool_from], 0) != cudaSuccess)
           return CSA_ERR_CUDA;
         uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
         hist_off += index_hist_bytes(&ix);
         if (run_index_decode(&ix, region, ls, h, ix.pool_out ? SS->pool[i] : nullptr) != cudaSuccess) return CSA_ERR_CUDA;
-      } else if (cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
+      } else if (L.mode == CSA_MODE_REUSE &&
+                 cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
         return CSA_ERR_CUDA;
       }
       if (cudaEventRecord(SS->idx[i], ls) != cudaSuccess) return CSA_ERR_CUDA;

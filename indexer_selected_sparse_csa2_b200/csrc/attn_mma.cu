@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "attn_tc.cuh"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -48,6 +49,8 @@ struct AttnParams {
   int n_splits;
   float* part_o;              // [B*n_q][n_splits][H][512]
   float* part_ml;             // [B*n_q][n_splits][H][2]
+  const float* rope_cs;       // optional [B*n_q][32][2]: partial RoPE of q, inverse on out
+  int out_bf16;               // out is bf16
 };
 
 constexpr int kAttnThreads = 256;
@@ -163,8 +166,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
   // Q (fp32) -> fp16 shared
   const float* qg = p.q + (int64_t)bt * H * kD;
   for (int i = tid; i < H * kD / 4; i += kAttnThreads) {
-    const float4 v = reinterpret_cast<const float4*>(qg)[i];
+    float4 v = reinterpret_cast<const float4*>(qg)[i];
     const int h = (4 * i) / kD, d = (4 * i) % kD;
+    if (p.rope_cs && d >= kRopeStart) {
+      const float4 k = *reinterpret_cast<const float4*>(p.rope_cs + (int64_t)bt * 64 + (d - kRopeStart));
+      const float2 r0 = rope_fwd(v.x, v.y, k.x, k.y), r1 = rope_fwd(v.z, v.w, k.z, k.w);
+      v = make_float4(r0.x, r0.y, r1.x, r1.y);
+    }
     __half2* dst = reinterpret_cast<__half2*>(Qs + h * kQStride + d);
     __half2* dlo = reinterpret_cast<__half2*>(Ql + h * kQStride + d);
     const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
@@ -345,13 +353,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
         p.lse[(int64_t)bt * H + h1] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
       }
     }
-    float* out0 = p.out + ((int64_t)bt * H + h0) * kD + d0;
-    float* out1 = p.out + ((int64_t)bt * H + h1) * kD + d0;
+    const float* cs = p.rope_cs ? p.rope_cs + (int64_t)bt * 64 : nullptr;
+    const int64_t o0 = ((int64_t)bt * H + h0) * kD + d0, o1 = ((int64_t)bt * H + h1) * kD + d0;
 #pragma unroll
     for (int nt = 0; nt < NT_O; ++nt) {
       const int d = 8 * nt + 2 * t4;
-      *reinterpret_cast<float2*>(out0 + d) = make_float2(o[nt][0] * sc0, o[nt][1] * sc0);
-      *reinterpret_cast<float2*>(out1 + d) = make_float2(o[nt][2] * sc1, o[nt][3] * sc1);
+      store_out2(p.out, p.out_bf16, o0 + d, rope_out2(make_float2(o[nt][0] * sc0, o[nt][1] * sc0), cs, d0 + d));
+      store_out2(p.out, p.out_bf16, o1 + d, rope_out2(make_float2(o[nt][2] * sc1, o[nt][3] * sc1), cs, d0 + d));
     }
   } else {
     const int64_t base = ((int64_t)bt * p.n_splits + split) * H;
@@ -443,8 +451,9 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p
       acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
     }
     const float inv = inv_s;
-    *reinterpret_cast<float4*>(p.out + ((int64_t)bt * H + h) * kD + d) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    const float* cs = p.rope_cs ? p.rope_cs + (int64_t)bt * 64 : nullptr;
+    store_out4(p.out, p.out_bf16, ((int64_t)bt * H + h) * kD + d,
+               rope_out4(make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv), cs, d));
   }
 }
 
@@ -532,6 +541,7 @@ static cudaError_t launch_attn_64_tc(AttnParams& p, const void* q2, cudaStream_t
   static_assert(kTileE == 64, "split boundaries must fall on 64-entry tiles");
   t.tiles_per_split = p.tiles_per_split;
   t.n_splits = p.n_splits; t.part_o = p.part_o; t.part_ml = p.part_ml;
+  t.rope_cs = p.rope_cs; t.out_bf16 = p.out_bf16;
   cudaError_t e = launch_attn_tc(t, stream);
   if (e != cudaSuccess) return e;
   if (p.n_splits > 1) {
@@ -558,6 +568,7 @@ cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t strea
   p.scale_log2 = a->softmax_scale * kLog2e;
   p.sink = a->sink;
   p.out = a->out; p.lse = a->lse;
+  p.rope_cs = a->rope_cs; p.out_bf16 = a->out_bf16 != 0;
   p.n_entries = a->K + a->n_win;
   p.tiles_per_split = pl.tiles_per_split;
   p.n_splits = pl.n_splits;

@@ -40,6 +40,7 @@
 #include "sm100.cuh"
 #include "q2.cuh"
 #include "attn_tc.cuh"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       if (i < 128 * 16) {
         const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
         uint32_t o[4];
+        rope_q8(f[2 * t], f[2 * t + 1], p.rope_cs ? p.rope_cs + (int64_t)bt * 64 : nullptr, 48 + 8 * kb + c8);
         q_hilo_perm8(f[2 * t], f[2 * t + 1], r & 1, o);
         *reinterpret_cast<uint4*>(S.q2 + kb * kAtQBlkBytes + sw128_offset_h(r, 8 * c8)) =
             make_uint4(o[0], o[1], o[2], o[3]);
@@ -603,9 +605,21 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
         for (int k = 0; k < 64; ++k) o[k] = 0u;
       }
       if (p.n_splits == 1) {
-        float* dst = p.out + (int64_t)bt * kAtH * kD + d;
 #pragma unroll
-        for (int hd = 0; hd < kAtH; ++hd) dst[(int64_t)hd * kD] = __uint_as_float(o[hd]) * S.scl[hd];
+        for (int hd = 0; hd < kAtH; ++hd) o[hd] = __float_as_uint(__uint_as_float(o[hd]) * S.scl[hd]);
+        if (p.rope_cs && c == 3 && qtr >= 2) {
+          // channels 448..511: channel d ^ 1 of the rotated pair sits in lane ^ 2
+          const float2 k = *reinterpret_cast<const float2*>(p.rope_cs + (int64_t)bt * 64 + ((d - kRopeStart) & ~1));
+#pragma unroll
+          for (int hd = 0; hd < kAtH; ++hd) {
+            const float v = __uint_as_float(o[hd]);
+            const float pv = __shfl_xor_sync(0xffffffffu, v, 2);
+            o[hd] = __float_as_uint((d & 1) ? v * k.x - pv * k.y : v * k.x + pv * k.y);
+          }
+        }
+        const int64_t base = (int64_t)bt * kAtH * kD + d;
+#pragma unroll
+        for (int hd = 0; hd < kAtH; ++hd) store_out1(p.out, p.out_bf16, base + (int64_t)hd * kD, __uint_as_float(o[hd]));
       } else {
         float* dst = p.part_o + ((int64_t)bt * p.n_splits + split) * kAtH * kD + d;
 #pragma unroll

@@ -26,6 +26,8 @@ struct AttnTcParams {
   const uint8_t* q2;          // optional: q already staged (q2.cuh layout), [B*n_q] tokens
   float* part_o;              // [B*n_q][n_splits][64][512] when n_splits > 1
   float* part_ml;             // [B*n_q][n_splits][64][2]
+  const float* rope_cs;       // optional [B*n_q][32][2] (cos, sin): partial RoPE of q, inverse on out
+  int out_bf16;               // out is bf16
 };
 
 cudaError_t launch_attn_tc(const AttnTcParams& p, cudaStream_t stream);

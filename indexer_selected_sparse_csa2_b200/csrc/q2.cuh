@@ -12,6 +12,7 @@
 // token (prologue) and every split CTA copies it instead of converting q.
 #pragma once
 #include "sm100.cuh"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -41,14 +42,17 @@ CSA_DEV void q_hilo_perm8(float4 a, float4 c, bool lo, uint32_t (&o)[4]) {
   }
 }
 
-// One warp stages head h of one token (q_tok: [64][512] fp32) into q2_tok.
-CSA_DEV void encode_q2_head(const float* q_tok, int h, int lane, uint8_t* q2_tok) {
+// One warp stages head h of one token (q_tok: [64][512] fp32) into q2_tok;
+// cs_tok: the token's optional [32][2] RoPE table (partial RoPE of channels
+// 448..511 before the hi / lo split).
+CSA_DEV void encode_q2_head(const float* q_tok, int h, int lane, uint8_t* q2_tok, const float* cs_tok) {
   const float4* src = reinterpret_cast<const float4*>(q_tok + (int64_t)h * 512 + 16 * lane);
   const float4 a0 = src[0], c0 = src[1], a1 = src[2], c1 = src[3];
 #pragma unroll
   for (int gg = 0; gg < 2; ++gg) {
     const int g = 2 * lane + gg;                  // channels 8g .. 8g + 7
-    const float4 a = gg ? a1 : a0, c = gg ? c1 : c0;
+    float4 a = gg ? a1 : a0, c = gg ? c1 : c0;
+    rope_q8(a, c, cs_tok, g);
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
       uint32_t o[4];

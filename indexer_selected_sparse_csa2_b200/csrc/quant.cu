@@ -43,11 +43,9 @@ CSA_DEV void load16(const void* row, int lane, float (&x)[16]) {
   }
 }
 
-// One warp encodes row `row` of the source into one FP4 entry.
-template <int SRC>
-CSA_DEV void encode_fp4_row(const void* row, int lane, uint8_t* out) {
-  float x[16];
-  load16<SRC>(row, lane, x);
+// Lane `lane` of a warp encodes channels [16 lane, 16 lane + 16) of one FP4
+// entry (one scale block) from values in registers.
+CSA_DEV void encode_fp4_vals(const float (&x)[16], int lane, uint8_t* out) {
   float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
@@ -64,6 +62,14 @@ CSA_DEV void encode_fp4_row(const void* row, int lane, uint8_t* out) {
   }
   *reinterpret_cast<uint2*>(out + 8 * lane) = make_uint2(packed[0], packed[1]);
   out[256 + lane] = (uint8_t)s_code;
+}
+
+// One warp encodes row `row` of the source into one FP4 entry.
+template <int SRC>
+CSA_DEV void encode_fp4_row(const void* row, int lane, uint8_t* out) {
+  float x[16];
+  load16<SRC>(row, lane, x);
+  encode_fp4_vals(x, lane, out);
 }
 
 template <int SRC>
@@ -127,12 +133,8 @@ __global__ void __launch_bounds__(256) quant_fp8w_kernel(const void* __restrict_
     encode_fp8w_row<SRC>(static_cast<const uint8_t*>(src) + r * src_stride_bytes, lane, dst + r * dst_stride);
 }
 
-// Plain E4M3 cast of 16 consecutive values (column group c of a row).
-template <int SRC>
-CSA_DEV void encode_plain16(const void* row, int c, uint8_t* out_row) {
-  float x[16];
-  // reuse the 16-value loader with "lane" = column group
-  load16<SRC>(row, c, x);
+// Plain E4M3 cast of 16 values in registers into column group c of a row.
+CSA_DEV void encode_plain_vals(const float (&x)[16], int c, uint8_t* out_row) {
   uint32_t w[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -141,6 +143,96 @@ CSA_DEV void encode_plain16(const void* row, int c, uint8_t* out_row) {
     w[i] = lo | (hi << 16);
   }
   *reinterpret_cast<uint4*>(out_row + 16 * c) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Plain E4M3 cast of 16 consecutive values (column group c of a row).
+template <int SRC>
+CSA_DEV void encode_plain16(const void* row, int c, uint8_t* out_row) {
+  float x[16];
+  // reuse the 16-value loader with "lane" = column group
+  load16<SRC>(row, c, x);
+  encode_plain_vals(x, c, out_row);
+}
+
+// ------------------------------------------------------------ compressor --
+// The m-token compressor of the encoder's CSA2 layers (DeepSeek-V4.1-Flash
+// architecture database, cache groups: one shared K=V entry per 2 tokens for
+// the encoder's main KV and indexer K, pooled with a gate in fp32; the
+// ratio-1 compressor is plain).  Per channel of a group of m token rows x_i
+// with gate logits g_i: w_i = exp(g_i - max_j g_j), entry = sum_i w_i x_i /
+// sum_i w_i, in fp32; then the entry is encoded like any cache row.  One
+// thread = 16 channels of one group (one FP4 scale block); token row r of
+// the source at src + r * src_stride_bytes, its gates at gate + r * gate_stride.
+template <int SRC>
+__global__ void __launch_bounds__(256) compress_kernel(const void* __restrict__ src, const float* __restrict__ gate,
+                                                       int64_t n_groups, int m, int dim, int64_t src_stride_bytes,
+                                                       int64_t gate_stride, int fmt, uint8_t* __restrict__ dst,
+                                                       int64_t dst_stride) {
+  pdl_enter();
+  const int per_row = dim >> 4;
+  const int64_t units = n_groups * per_row;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < units; u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = u / per_row;
+    const int c = (int)(u - n * per_row);
+    float x[16];
+    if (m == 1) {
+      load16<SRC>(static_cast<const uint8_t*>(src) + n * src_stride_bytes, c, x);
+    } else {
+      float gmax[16], acc[16], wsum[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) { gmax[k] = -INFINITY; acc[k] = 0.f; wsum[k] = 0.f; }
+      for (int i = 0; i < m; ++i) {
+        const float4* gp = reinterpret_cast<const float4*>(gate + (n * m + i) * gate_stride + 16 * c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 g = gp[q];
+          gmax[4 * q] = fmaxf(gmax[4 * q], g.x); gmax[4 * q + 1] = fmaxf(gmax[4 * q + 1], g.y);
+          gmax[4 * q + 2] = fmaxf(gmax[4 * q + 2], g.z); gmax[4 * q + 3] = fmaxf(gmax[4 * q + 3], g.w);
+        }
+      }
+      for (int i = 0; i < m; ++i) {
+        float xi[16];
+        load16<SRC>(static_cast<const uint8_t*>(src) + (n * m + i) * src_stride_bytes, c, xi);
+        const float4* gp = reinterpret_cast<const float4*>(gate + (n * m + i) * gate_stride + 16 * c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 g = gp[q];
+          const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float w = expf(gg[k] - gmax[4 * q + k]);
+            acc[4 * q + k] = fmaf(w, xi[4 * q + k], acc[4 * q + k]);
+            wsum[4 * q + k] += w;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) x[k] = __fdiv_rn(acc[k], wsum[k]);
+    }
+    if (fmt == CSA_FMT_FP4_E2M1_E4M3X16) encode_fp4_vals(x, c, dst + n * dst_stride);
+    else encode_plain_vals(x, c, dst + n * dst_stride);
+  }
+}
+
+cudaError_t launch_compress(const void* src, int src_dtype, const float* gate, int64_t n_groups, int m, int dim,
+                            int64_t src_row_stride, int64_t gate_row_stride, int fmt, void* dst,
+                            int64_t dst_row_stride, cudaStream_t stream) {
+  const int64_t esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  const int64_t units = n_groups * (dim >> 4);
+  int64_t g = (units + 255) / 256;
+  if (g > kNumSMs * 8) g = kNumSMs * 8;
+  if (g < 1) g = 1;
+  // a group's rows are m consecutive token rows of src_row_stride elements
+  const int64_t stride_b = src_row_stride * esz;
+  ProfScope ps(stream, "compress");
+  if (src_dtype == CSA_SRC_BF16)
+    launch_k(compress_kernel<1>, dim3((unsigned)g), dim3(256), 0, stream, src, gate, n_groups, m, dim, stride_b,
+             gate_row_stride, fmt, static_cast<uint8_t*>(dst), dst_row_stride);
+  else
+    launch_k(compress_kernel<0>, dim3((unsigned)g), dim3(256), 0, stream, src, gate, n_groups, m, dim, stride_b,
+             gate_row_stride, fmt, static_cast<uint8_t*>(dst), dst_row_stride);
+  note_launches(1);
+  return cudaGetLastError();
 }
 
 // Plain E4M3 cast: each thread encodes 16 consecutive values of one row.
@@ -190,7 +282,7 @@ __global__ void __launch_bounds__(256) quant_batch_kernel(QuantBatch qb) {
     } else if (J.fmt == kFmtStageQ2) {
       const int64_t tok = lu >> 6;
       encode_q2_head(reinterpret_cast<const float*>(src) + tok * (64 * 512), (int)(lu & 63), lane,
-                     J.dst + tok * kQ2TokenBytes);
+                     J.dst + tok * kQ2TokenBytes, J.aux ? J.aux + tok * 64 : nullptr);
     } else {
       const int per_row = J.dim >> 4;
       const int64_t g = lu * 32 + lane;

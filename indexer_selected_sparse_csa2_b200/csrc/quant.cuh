@@ -21,6 +21,7 @@ struct QuantBatchJob {
   int bf16;                // source is bf16 (else fp32)
   int dim;
   int64_t unit0;           // first warp unit of this job in the flat list
+  const float* aux;        // query staging: optional [tokens][32][2] RoPE (cos, sin) table
 };
 
 struct QuantBatch {

@@ -16,6 +16,12 @@ Readings used here:
               a new Top-K (inside the pool when one is named), own window.
     Reuse   - the Top-K indices of the named earlier layer, its owner's main
               KV, its own window and attention queries; no scoring.
+    SWA     - a sliding-window layer: attention over its own window alone
+              (the stack's first two layers, architecture database layer
+              pattern "2 SWA + 18 CSA2 m=2 + 20 CSA2 m=1").
+An owner whose caches hold one entry per m tokens (the encoder's CSA2 m=2
+layers) has owner_len(owner) = floor(T / m) entries, and its layers select
+among those entries; windows stay per token.
 Query t of a sequence with n_q new tokens and cache length T sits at position
 T - n_q + t and sees positions [0, T - n_q + t] (decode: n_q = 1, all of
 [0, T)); its window rows are [t, t + n_win) of the layer's window buffer.
@@ -32,7 +38,7 @@ from .mxfp4 import mx_index_scores
 from .attention import attend
 from .quant import fp4_dequant_rows, fp8_window_dequant_rows
 
-FULL, REINDEX, REUSE = 0, 1, 2
+FULL, REINDEX, REUSE, SWA = 0, 1, 2, 3
 
 
 @dataclass
@@ -61,7 +67,8 @@ def run_stack(layers: Sequence, T: int, n_q: int, K: int, n_win: int, scale: flo
               inputs: Callable[[int], LayerInputs],
               queries: Optional[Sequence[int]] = None,
               pool_blocks: int = 2048, pool_block_len: int = 8,
-              keep_scores: bool = False, key_format: str = "e4m3") -> List[LayerResult]:
+              keep_scores: bool = False, key_format: str = "e4m3",
+              owner_len: Optional[Callable[[int], int]] = None) -> List[LayerResult]:
     """Run a layer stack for one sequence.
 
     ``layers``: objects with mode / owner / reuse_from / build_pool / pool_from.
@@ -78,13 +85,18 @@ def run_stack(layers: Sequence, T: int, n_q: int, K: int, n_win: int, scale: flo
         inp = inputs(li)
         idx_rows, scores_rows = [], []
         pool, pool_len = None, 0
-        if L.mode == REUSE:
+        T_o = T if owner_len is None or L.mode == SWA else owner_len(L.owner)
+        if T_o != T:
+            assert n_q == 1, "compressed caches are read at decode"
+        if L.mode == SWA:
+            idx_rows = [np.full(K, -1, dtype=np.int32) for _ in qs]
+        elif L.mode == REUSE:
             src = results[L.reuse_from]
             idx_rows = list(src.idx)
         else:
             kc = keys(L.owner)
             for t in qs:
-                n_t = T - n_q + t + 1
+                n_t = T_o - n_q + t + 1
                 if L.mode == REINDEX and L.pool_from >= 0:
                     P = results[L.pool_from]
                     ppos = P.pool[:P.pool_len].astype(np.int64)

@@ -68,3 +68,22 @@ def oracle_attend_on(case, cfg, li, t, idx_row, inputs=None):
     Xm = fp4_dequant_rows(case.main_entries(L.owner, sel)) if sel.size else np.zeros((0, 512))
     Xw = fp8_window_dequant_rows(inp.window[t:t + cfg.n_win])
     return attend(inp.q[t], np.concatenate([Xm, Xw], axis=0), cfg.softmax_scale, inp.sink)
+
+
+BF16_HALF_ULP = 2.0 ** -8
+
+
+def assert_close_bf16(gpu, ora, what=""):
+    """bf16 outputs: the fp32 rule plus the bf16 rounding of the result (at most
+    half an ulp, 2^-8 relative), since the cast may round either way of a
+    result that is itself within the fp32 tolerance."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ora = np.asarray(ora, dtype=np.float64)
+    assert gpu.shape == ora.shape, (gpu.shape, ora.shape)
+    err = np.abs(gpu - ora)
+    bound = ATOL + (RTOL + BF16_HALF_ULP) * np.abs(ora)
+    bad = ~(err <= bound)
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(bad, err - bound, -np.inf)), bad.shape)
+        raise AssertionError(f"{what}: {bad.sum()} elements out of tolerance; worst at {i}: "
+                             f"gpu={gpu[i]!r} oracle={ora[i]!r}")
