@@ -87,3 +87,53 @@ def assert_close_bf16(gpu, ora, what=""):
         i = np.unravel_index(np.argmax(np.where(bad, err - bound, -np.inf)), bad.shape)
         raise AssertionError(f"{what}: {bad.sum()} elements out of tolerance; worst at {i}: "
                              f"gpu={gpu[i]!r} oracle={ora[i]!r}")
+
+
+BOUNDARY_REL = 1e-5
+
+
+def check_codes_near_boundaries(gpu_bytes, exact, kind, what=""):
+    """Encodings of values that pass through fp32 arithmetic the oracle does in
+    float64 (the compressor's exp and division): a GPU code may differ from
+    the oracle's only where the exact value lies within BOUNDARY_REL of the
+    rounding midpoint between the two codes' values.  kind: "fp4" (288-byte
+    entries of 512 channels) or "e4m3" (plain codes).  Returns the number of
+    differing codes."""
+    from oracle import codecs, quant
+    exact = np.asarray(exact, dtype=np.float64)
+    gpu_bytes = np.asarray(gpu_bytes, dtype=np.uint8)
+    if kind == "e4m3":
+        ora = quant.e4m3_cast(exact.astype(np.float32))
+        diff = gpu_bytes != ora
+        if diff.any():
+            mid = (codecs.e4m3_decode(gpu_bytes[diff]) + codecs.e4m3_decode(ora[diff])) / 2
+            x = exact[diff]
+            assert np.all(np.abs(x - mid) <= BOUNDARY_REL * np.maximum(np.abs(x), 2.0 ** -9)), what
+        return int(diff.sum())
+    assert kind == "fp4"
+    ora = quant.fp4_quant_rows(exact.astype(np.float32))
+    n_diff = 0
+    for r in range(exact.shape[0]):
+        if np.array_equal(gpu_bytes[r], ora[r]):
+            continue
+        for blk in range(32):
+            xs = exact[r, 16 * blk:16 * blk + 16]
+            sg, so = gpu_bytes[r, 256 + blk], ora[r, 256 + blk]
+            if sg != so:
+                # the block scale itself sits at a rounding boundary of amax / 6
+                a6 = np.abs(xs).max() / 6
+                mid = (codecs.e4m3_decode(np.array([sg])) + codecs.e4m3_decode(np.array([so])))[0] / 2
+                assert abs(a6 - mid) <= BOUNDARY_REL * a6, f"{what} row {r} block {blk} scale"
+                n_diff += 16
+                continue
+            s = codecs.e4m3_decode(np.array([sg]))[0]
+            for c in range(16):
+                b = 8 * blk + c // 2
+                cg = (gpu_bytes[r, b] >> (4 * (c % 2))) & 0xF
+                co = (ora[r, b] >> (4 * (c % 2))) & 0xF
+                if cg != co:
+                    mid = (codecs.e2m1_decode(np.array([cg])) + codecs.e2m1_decode(np.array([co])))[0] / 2
+                    v = xs[c] / s
+                    assert abs(v - mid) <= BOUNDARY_REL * max(abs(v), 0.5), f"{what} row {r} ch {16 * blk + c}"
+                    n_diff += 1
+    return n_diff
