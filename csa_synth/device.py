@@ -46,31 +46,38 @@ class DeviceCase:
                  keep_scores: bool = False, batches: Optional[List[int]] = None):
         import torch
         csa = _lib()
-        if cfg.key_format != "e4m3":
+        if cfg.key_format not in ("e4m3", "mxfp4"):
             raise NotImplementedError(f"indexer key format {cfg.key_format!r} has no device encoder")
         self.cfg = cfg
         self.device = device
         B, T = cfg.B, cfg.T
         self.keys: Dict[int, object] = {}
+        self.key_scales: Dict[int, object] = {}     # MXFP4 keys: exponent bytes [B, T, d_I / 32]
         self.kv: Dict[int, object] = {}
+        mx = cfg.key_format == "mxfp4"
         for o in cfg.owners:
             E, m = cfg.entries(o), cfg.ratio(o)
-            keys = torch.empty((B, E, cfg.d_I), dtype=torch.uint8, device=device)
+            keys = torch.empty((B, E, cfg.d_I // 2 if mx else cfg.d_I), dtype=torch.uint8, device=device)
+            if mx:
+                self.key_scales[o] = torch.empty((B, E, cfg.d_I // 32), dtype=torch.uint8, device=device)
             kv = torch.empty((B, E, csa.FP4_ENTRY_BYTES), dtype=torch.uint8, device=device)
             for b in range(B):
                 for e0 in range(0, E, UPLOAD_ROWS):
                     n = min(UPLOAD_ROWS, E - e0)
                     kx = torch.from_numpy(wl.index_key(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
-                    mx = self._latent_tensor(wl.main_latent(cfg, o, b, e0 * m, n * m, threads=threads))
+                    lx = self._latent_tensor(wl.main_latent(cfg, o, b, e0 * m, n * m, threads=threads))
                     if m == 1:
-                        csa.csa_quant_kv(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, e0:e0 + n])
-                        csa.csa_quant_kv(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
+                        if o in self.key_scales:
+                            csa.csa_quant_mxfp4(kx, keys[b, e0:e0 + n], self.key_scales[o][b, e0:e0 + n])
+                        else:
+                            csa.csa_quant_kv(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, e0:e0 + n])
+                        csa.csa_quant_kv(lx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
                     else:
                         # the compressor pools each group of m token rows into one entry
                         kg = torch.from_numpy(wl.index_gate(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
                         mg = torch.from_numpy(wl.main_gate(cfg, o, b, e0 * m, n * m, threads=threads)).to(device)
                         csa.csa_compress_kv(kx, kg, m, csa.CSA_FMT_FP8_E4M3_PLAIN, keys[b, e0:e0 + n])
-                        csa.csa_compress_kv(mx, mg, m, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
+                        csa.csa_compress_kv(lx, mg, m, csa.CSA_FMT_FP4_E2M1_E4M3X16, kv[b, e0:e0 + n])
             self.keys[o] = keys
             self.kv[o] = kv
         self.layers: List[DeviceLayer] = []
@@ -152,7 +159,8 @@ class DeviceCase:
                         kvrow, krow = self.kv[o][0, t_new:], self.keys[o][0, t_new:]
                         kv_stride, k_stride = self.kv[o].stride(1), self.keys[o].stride(1)
                     jobs.append(csa.quant_job(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kvrow, kv_stride))
-                    jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, k_stride))
+                    if cfg.key_format == "e4m3":       # (MXFP4 keys are encoded whole above)
+                        jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, k_stride))
                     self._append_src += [mx, kx]
                 r0 = cfg.win_rows - n_new
                 if n_new == 1:
@@ -168,7 +176,8 @@ class DeviceCase:
                     d.append[k] = j
             if L.mode in (FULL, REINDEX):
                 d.index = csa.index_args(
-                    keys=self.keys[o], q=dl.qI, w=dl.w, K=cfg.K, idx=dl.idx, T=cfg.entries(o), n_q=cfg.n_q,
+                    keys=self.keys[o], key_scales=self.key_scales.get(o), q=dl.qI, w=dl.w, K=cfg.K, idx=dl.idx,
+                    T=cfg.entries(o), n_q=cfg.n_q,
                     pool_out=dl.pool, pool_out_len=dl.pool_len, pool_blocks=cfg.pool_blocks,
                     pool_block_len=cfg.pool_block_len, scores=dl.scores)
             d.attn = csa.attn_args(q=dl.q, kv=self.kv[o] if L.mode != SWA else None, idx=None, win=dl.win,

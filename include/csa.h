@@ -151,7 +151,33 @@ typedef struct {
   float* scores;             /* optional out (decode only): fp32 scores
                                 [B][T] (or [B][pool_cap] when searching a
                                 pool; slots past pool_len are not written) */
+  /* Indexer-key format.  CSA_KEY_E4M3: plain E4M3 keys (d_I = 64, H_I <= 8,
+   * the fields below unused).  CSA_KEY_MXFP4: the pages' MXFP4 keys
+   * (architecture database, indexer K: E2M1 with one E8M0 scale per 32
+   * channels; techniques map: 32 heads x 128): d_I = 128, H_I = 32, decode
+   * scans only (no pool search); `keys` holds the E2M1 codes (64 bytes per
+   * key, even channel in the low nibble) and `key_scales` the 4 exponent
+   * bytes (e + 127, block order) of key s at key_scales +
+   * b*key_scale_batch_stride + s*key_scale_row_stride (strides multiples of
+   * 4).  Block b of the key contributes 2^e_b * <q block b, E2M1 codes>. */
+  int32_t key_format;
+  const uint8_t* key_scales;
+  int64_t key_scale_row_stride;
+  int64_t key_scale_batch_stride;
 } csa_index_args;
+
+typedef enum { CSA_KEY_E4M3 = 0, CSA_KEY_MXFP4 = 1 } csa_key_format;
+
+/* MXFP4 encoding of indexer keys into the two planes above: per block of 32
+ * channels, e = the smallest integer with amax <= 6 * 2^e, clamped to
+ * [-127, 127] (amax = 0 -> -127); codes E2M1_rne_sat(x * 2^-e).
+ * src: n_rows rows of `dim` (a multiple of 32) fp32 / bf16 values, row r at
+ * src + r * src_row_stride elements; codes row r at codes + r *
+ * codes_row_stride (dim / 2 bytes), exponent bytes at scales + r *
+ * scales_row_stride (dim / 32 bytes). */
+csa_status csa_quant_mxfp4(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim, int64_t src_row_stride,
+                           uint8_t* codes, int64_t codes_row_stride, uint8_t* scales, int64_t scales_row_stride,
+                           csa_stream_t stream);
 
 size_t csa_index_workspace_size(const csa_index_args* a);
 csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t workspace_bytes,

@@ -34,6 +34,7 @@ CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_SHAPE, CSA_ERR_ALIGNMENT, CSA_ERR_UNSUPPORT
 CSA_SRC_F32, CSA_SRC_BF16 = 0, 1
 CSA_FMT_FP4_E2M1_E4M3X16, CSA_FMT_FP8_E4M3_UE8M0X32, CSA_FMT_FP8_E4M3_PLAIN = 0, 1, 2
 CSA_MODE_FULL, CSA_MODE_REINDEX, CSA_MODE_REUSE, CSA_MODE_SWA = 0, 1, 2, 3
+CSA_KEY_E4M3, CSA_KEY_MXFP4 = 0, 1
 FP4_ENTRY_BYTES, FP8_ENTRY_BYTES = 288, 528
 
 _p = ctypes.c_void_p
@@ -48,7 +49,9 @@ class IndexArgs(ctypes.Structure):
                 ("q", _p), ("w", _p), ("K", _i32),
                 ("pool", _p), ("pool_len", _p), ("pool_cap", _i32),
                 ("pool_out", _p), ("pool_out_len", _p), ("pool_blocks", _i32), ("pool_block_len", _i32),
-                ("idx", _p), ("scores", _p)]
+                ("idx", _p), ("scores", _p),
+                ("key_format", _i32), ("key_scales", _p), ("key_scale_row_stride", _i64),
+                ("key_scale_batch_stride", _i64)]
 
 
 class AttnArgs(ctypes.Structure):
@@ -82,6 +85,7 @@ def _sig(name, res, args):
 
 
 _quant = _sig("csa_quant_kv", _i32, [_p, _i32, _i64, _i32, _i64, _i32, _p, _i64, _p])
+_quant_mx = _sig("csa_quant_mxfp4", _i32, [_p, _i32, _i64, _i32, _i64, _p, _i64, _p, _i64, _p])
 _compress = _sig("csa_compress_kv", _i32, [_p, _i32, _p, _i64, _i32, _i32, _i64, _i64, _i32, _p, _i64, _p])
 _index_ws = _sig("csa_index_workspace_size", ctypes.c_size_t, [ctypes.POINTER(IndexArgs)])
 _index = _sig("csa_index_topk", _i32, [ctypes.POINTER(IndexArgs), _p, ctypes.c_size_t, _p])
@@ -109,7 +113,7 @@ _cp_merge = _sig("csa_cp_merge_topk", _i32, [_p, _p, _i32, _i32, _i32, _i32, _p,
 _cp_localize = _sig("csa_cp_localize", _i32, [_p, _i32, _i32, _i64, _i64, _p, _p])
 _cp_combine = _sig("csa_cp_combine", _i32, [_p, _p, _i32, _i32, _i32, _p, _p, _p, _p])
 
-EXPORTED = ["csa_quant_kv", "csa_compress_kv", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
+EXPORTED = ["csa_quant_kv", "csa_compress_kv", "csa_quant_mxfp4", "csa_index_workspace_size", "csa_index_topk", "csa_topk_workspace_size",
             "csa_topk_scores", "csa_attn_workspace_size", "csa_sparse_attn", "csa_layer_workspace_size",
             "csa_layer_step", "csa_status_string", "csa_launch_count", "csa_version",
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
@@ -208,6 +212,16 @@ def csa_quant_kv(src, fmt: int, dst, n_rows: Optional[int] = None, dim: Optional
     dst_row_stride = dst.stride(0) * dst.element_size() if dst_row_stride is None else dst_row_stride
     _check(_quant(_ptr(src), dtype, n_rows, dim, src_row_stride, fmt, _ptr(dst), dst_row_stride,
                   _stream(stream)), "csa_quant_kv")
+
+
+def csa_quant_mxfp4(src, codes, scales, stream=None) -> None:
+    """MXFP4 encoding of ``src`` (fp32 / bf16 [n_rows, dim]) into ``codes``
+    (uint8 [n_rows, dim/2]) and ``scales`` (uint8 [n_rows, dim/32])."""
+    torch = _torch()
+    dtype = CSA_SRC_BF16 if src.dtype == torch.bfloat16 else CSA_SRC_F32
+    _check(_quant_mx(_ptr(src), dtype, src.shape[0], src.shape[-1], src.stride(0), _ptr(codes),
+                     codes.stride(0) * codes.element_size(), _ptr(scales), scales.stride(0) * scales.element_size(),
+                     _stream(stream)), "csa_quant_mxfp4")
 
 
 def csa_compress_kv(src, gate, m: int, fmt: int, dst, dst_row_stride: Optional[int] = None, stream=None) -> None:
@@ -344,9 +358,10 @@ def csa_cp_combine(o_parts, lse_parts, out, lse=None, sink=None, stream=None) ->
 # ------------------------------------------------------- argument builders --
 def index_args(*, keys, q, w, K: int, idx, T: Optional[int] = None, n_q: int = 1,
                pool=None, pool_len=None, pool_out=None, pool_out_len=None,
-               pool_blocks: int = 2048, pool_block_len: int = 8, scores=None) -> IndexArgs:
+               pool_blocks: int = 2048, pool_block_len: int = 8, scores=None, key_scales=None) -> IndexArgs:
     """IndexArgs from torch tensors: keys uint8 [B, T, 64] (any row / batch stride),
-    q uint8 [B, n_q, H_I, 64], w fp32 [B, n_q, H_I], idx int32 [B, n_q, K]."""
+    q uint8 [B, n_q, H_I, d_I], w fp32 [B, n_q, H_I], idx int32 [B, n_q, K].
+    With key_scales (uint8 [B, T, 4]) the keys are MXFP4 codes (d_I = 128)."""
     B = keys.shape[0]
     a = IndexArgs()
     a.B, a.n_q = B, n_q
@@ -361,8 +376,12 @@ def index_args(*, keys, q, w, K: int, idx, T: Optional[int] = None, n_q: int = 1
     a.pool_blocks, a.pool_block_len = pool_blocks, pool_block_len
     a.idx = _ptr(idx)
     a.scores = _ptr(scores)
+    if key_scales is not None:
+        a.key_format = CSA_KEY_MXFP4
+        a.key_scales = _ptr(key_scales)
+        a.key_scale_row_stride, a.key_scale_batch_stride = key_scales.stride(1), key_scales.stride(0)
     # the struct holds raw device pointers: keep the tensors alive with it
-    a._keep = (keys, q, w, pool, pool_len, pool_out, pool_out_len, idx, scores)
+    a._keep = (keys, q, w, pool, pool_len, pool_out, pool_out_len, idx, scores, key_scales)
     return a
 
 

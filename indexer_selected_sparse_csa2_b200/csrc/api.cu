@@ -23,6 +23,10 @@ void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_
 
 cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
                          int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream);
+cudaError_t launch_quant_mx(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
+                            uint8_t* codes, int64_t codes_row_stride, uint8_t* scales, int64_t scales_row_stride,
+                            cudaStream_t stream);
+int read_mx_error(bool clear);
 cudaError_t launch_compress(const void* src, int src_dtype, const float* gate, int64_t n_groups, int m, int dim,
                             int64_t src_row_stride, int64_t gate_row_stride, int fmt, void* dst,
                             int64_t dst_row_stride, cudaStream_t stream);
@@ -65,10 +69,21 @@ static csa_status check_quant(const void* src, int32_t src_dtype, int64_t n_rows
 static csa_status check_index(const csa_index_args* a) {
   if (!a) return CSA_ERR_INVALID_ARG;
   if (a->B < 1 || a->n_q < 1 || a->T < a->n_q || a->T >= ((int64_t)1 << 31)) return CSA_ERR_SHAPE;
-  if (a->H_I < 1 || a->H_I > 8 || a->d_I != kDI) return CSA_ERR_SHAPE;
+  if (a->key_format == CSA_KEY_MXFP4) {
+    if (a->H_I != 32 || a->d_I != 128) return CSA_ERR_SHAPE;
+    if (a->n_q != 1 || a->pool) return CSA_ERR_UNSUPPORTED;
+    if (!a->key_scales) return CSA_ERR_INVALID_ARG;
+    if (a->key_scale_row_stride < 4 || ((uintptr_t)a->key_scales & 3) || (a->key_scale_row_stride & 3) ||
+        (a->key_scale_batch_stride & 3))
+      return CSA_ERR_ALIGNMENT;
+  } else if (a->key_format != CSA_KEY_E4M3) {
+    return CSA_ERR_INVALID_ARG;
+  } else if (a->H_I < 1 || a->H_I > 8 || a->d_I != kDI) {
+    return CSA_ERR_SHAPE;
+  }
   if (a->K < 1 || a->K > 65536) return CSA_ERR_SHAPE;
   if (!a->keys || !a->q || !a->w || !a->idx) return CSA_ERR_INVALID_ARG;
-  if (a->key_row_stride < kDI) return CSA_ERR_SHAPE;
+  if (a->key_row_stride < (a->key_format == CSA_KEY_MXFP4 ? 64 : kDI)) return CSA_ERR_SHAPE;
   if (!al16(a->keys) || !al16i(a->key_row_stride) || !al16i(a->key_batch_stride) || !al16(a->q))
     return CSA_ERR_ALIGNMENT;
   if (a->n_q > 1) {
@@ -144,6 +159,21 @@ csa_status csa_compress_kv(const void* src, int32_t src_dtype, const float* gate
   if (m > 1 && (!al16(gate) || !al16i(gate_row_stride * 4))) return CSA_ERR_ALIGNMENT;
   return from_cuda(launch_compress(src, src_dtype, gate, n_groups, m, dim, src_row_stride, gate_row_stride, fmt, dst,
                                    dst_row_stride, (cudaStream_t)stream));
+}
+
+csa_status csa_quant_mxfp4(const void* src, int32_t src_dtype, int64_t n_rows, int32_t dim, int64_t src_row_stride,
+                           uint8_t* codes, int64_t codes_row_stride, uint8_t* scales, int64_t scales_row_stride,
+                           csa_stream_t stream) {
+  if (src_dtype != CSA_SRC_F32 && src_dtype != CSA_SRC_BF16) return CSA_ERR_INVALID_ARG;
+  if (n_rows < 0 || dim <= 0 || dim % 32) return CSA_ERR_SHAPE;
+  if (n_rows == 0) return CSA_OK;
+  if (!src || !codes || !scales) return CSA_ERR_INVALID_ARG;
+  if (src_row_stride < dim || (n_rows > 1 && (codes_row_stride < dim / 2 || scales_row_stride < dim / 32)))
+    return CSA_ERR_SHAPE;
+  const int64_t esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  if (!al16(src) || !al16i(src_row_stride * esz) || !al16(codes) || !al16i(codes_row_stride)) return CSA_ERR_ALIGNMENT;
+  return from_cuda(launch_quant_mx(src, src_dtype, n_rows, dim, src_row_stride, codes, codes_row_stride, scales,
+                                   scales_row_stride, (cudaStream_t)stream));
 }
 
 size_t csa_index_workspace_size(const csa_index_args* a) {
@@ -534,8 +564,8 @@ const char* csa_status_string(int32_t s) {
 
 int32_t csa_device_status(void) {
   const int a = read_tc_error(true), b = read_pf_error(true), c = read_at_error(true);
-  const int d = read_pk_error(true);
-  return (int32_t)(a ? a : (b ? b : (c ? c : d)));
+  const int d = read_pk_error(true), e = read_mx_error(true);
+  return (int32_t)(a ? a : (b ? b : (c ? c : (d ? d : e))));
 }
 
 uint64_t csa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -318,6 +318,76 @@ static int grid_for(int64_t work, int per_block) {
   return (int)(g < 1 ? 1 : (g > cap ? cap : g));
 }
 
+// ------------------------------------------------------------------ MXFP4 --
+// MXFP4 indexer keys (DeepSeek-V4.1-Flash architecture database, storage of
+// the indexer K groups: 4-bit E2M1 elements with one E8M0 scale per 32
+// channels, 68 bytes per 128-channel entry).  Per block of 32 channels: e is
+// the smallest integer with amax <= 6 * 2^e, clamped to [-127, 127] (amax = 0
+// -> -127), and code_i = E2M1_rne_sat(x_i * 2^-e) (an exact power-of-two
+// scaling unless the product underflows, where E2M1 gives +-0 anyway).  Codes
+// go to a code plane (two per byte, even channel in the low nibble), the
+// exponent bytes (e + 127) to a scale plane.
+// 6 = 1.5 * 2^2: for amax = f * 2^E with f in [1, 2), e = E - 2 when f <= 1.5
+// and E - 1 otherwise.
+CSA_DEV int mx_exponent(float amax) {
+  const uint32_t u = __float_as_uint(amax);
+  const int ef = (int)((u >> 23) & 0xFF);
+  if (ef == 0) return -127;  // zero or subnormal: 6 * 2^-127 >= amax
+  const uint32_t m = u & 0x7FFFFFu;
+  const int e = (ef - 127) - 2 + (m > 0x400000u ? 1 : 0);
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// One thread encodes 32 channels (one scale block) of one row.
+template <int SRC>
+__global__ void __launch_bounds__(256) quant_mx_kernel(const void* __restrict__ src, int64_t n_rows, int dim,
+                                                       int64_t src_stride_bytes, uint8_t* __restrict__ codes,
+                                                       int64_t codes_stride, uint8_t* __restrict__ scales,
+                                                       int64_t scales_stride) {
+  pdl_enter();
+  const int per_row = dim >> 5;
+  const int64_t total = n_rows * per_row;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < total; g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = g / per_row;
+    const int blk = (int)(g - r * per_row);
+    const uint8_t* row = static_cast<const uint8_t*>(src) + r * src_stride_bytes;
+    float x[32];
+    load16<SRC>(row, 2 * blk, *reinterpret_cast<float(*)[16]>(x));
+    load16<SRC>(row, 2 * blk + 1, *reinterpret_cast<float(*)[16]>(x + 16));
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const int e = mx_exponent(amax);
+    const float sc = pow2f(-e);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      // even channel in the low nibble
+      const uint32_t b = enc_e2m1x2(x[2 * i + 1] * sc, x[2 * i] * sc);
+      w[i >> 2] |= b << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint4*>(codes + r * codes_stride + 16 * blk) = make_uint4(w[0], w[1], w[2], w[3]);
+    scales[r * scales_stride + blk] = (uint8_t)(e + 127);
+  }
+}
+
+cudaError_t launch_quant_mx(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
+                            uint8_t* codes, int64_t codes_row_stride, uint8_t* scales, int64_t scales_row_stride,
+                            cudaStream_t stream) {
+  if (n_rows == 0) return cudaSuccess;
+  const int esz = src_dtype == CSA_SRC_BF16 ? 2 : 4;
+  const int g = grid_for(n_rows * (dim / 32), 256);
+  ProfScope ps(stream, "quant_mxfp4");
+  if (src_dtype == CSA_SRC_F32)
+    launch_k(quant_mx_kernel<0>, dim3(g), dim3(256), 0, stream, src, n_rows, dim, src_row_stride * esz, codes,
+             codes_row_stride, scales, scales_row_stride);
+  else
+    launch_k(quant_mx_kernel<1>, dim3(g), dim3(256), 0, stream, src, n_rows, dim, src_row_stride * esz, codes,
+             codes_row_stride, scales, scales_row_stride);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant(const void* src, int src_dtype, int64_t n_rows, int dim, int64_t src_row_stride,
                          int fmt, void* dst, int64_t dst_row_stride, cudaStream_t stream) {
   if (n_rows == 0) return cudaSuccess;
