@@ -147,13 +147,16 @@ def _algorithmic_bytes(cfg):
 
 KERNEL_SOURCES = {
     "index_score_tc[full]": "index_tc.cu",
+    "index_score_mx": "index_mx.cu",
     "index_score_decode[pool]": "index_decode.cu",
     "sparse_attn_tc": "attn_tc.cu",
     "attn_combine": "attn_mma.cu",
-    "select_extract": "select.cu",
-    "select_final": "select.cu",
-    "select_small": "select.cu",
+    "pool_select": "select_cluster.cu",
+    "pool_gather_select": "select_cluster.cu",
+    "pool_score_select": "select_cluster.cu",
+    "topk_select": "select_cluster.cu",
     "quant_batch": "quant.cu",
+    "quant_fp4": "quant.cu",
 }
 
 
@@ -183,18 +186,21 @@ def kernel_work(cfg):
     """Algorithmic HBM bytes and flops per launch of the decode step's kernels
     (what the kernel must read or write, and the multiply-adds x 2 it must do):
     * full scorer: B*T keys of 64 B; 2*64*H_I flops per (key, head);
-    * pool scorer: B*pool keys of 64 B (one Reindex layer per launch);
+    * pool select: the B*T/8 block maxima (4 B each) it reads;
+    * pool layer score + select: B*pool keys of 64 B (one Reindex layer per launch);
+    * the Full layer's select inside its pool: B*pool scores gathered (4 B);
     * attention: B*(K*288 + W*528) entry bytes; 2 * 2*H*512 flops per entry
       (logits and the weighted sum), one layer per launch;
-    * selects and the split combine: the scores / partials they read."""
+    * split combine: the partial O it reads (B * splits * H * 512 * 4 B)."""
     B, T, K, W, H, HI = cfg.B, cfg.T, cfg.K, cfg.n_win, cfg.H, cfg.H_I
     n_pool = cfg.pool_blocks * cfg.pool_block_len
+    nb = (T + cfg.pool_block_len - 1) // cfg.pool_block_len
     return {
         "index_score_tc[full]": {"bytes": B * T * 64, "flops": 2.0 * B * T * HI * 64, "engine": "fp8"},
-        "index_score_decode[pool]": {"bytes": B * n_pool * 64, "flops": 2.0 * B * n_pool * HI * 64, "engine": "fp8"},
+        "pool_select": {"bytes": B * nb * 4, "flops": 0.0, "engine": None},
+        "pool_score_select": {"bytes": B * n_pool * 64, "flops": 2.0 * B * n_pool * HI * 64, "engine": "fp8"},
+        "pool_gather_select": {"bytes": B * n_pool * 4, "flops": 0.0, "engine": None},
         "sparse_attn_tc": {"bytes": B * (K * 288 + W * 528), "flops": 4.0 * B * H * 512 * (K + W), "engine": "bf16"},
-        "select_extract": {"bytes": B * T * 4, "flops": 0.0, "engine": None},
-        "select_small": {"bytes": B * n_pool * 4, "flops": 0.0, "engine": None},
     }
 
 
@@ -485,7 +491,6 @@ def run_gpu(args, cfg, rank, world, local_rank):
     clocks.start()
     timed(run_step, starts, ends, False)
     barrier()
-    clk = clocks.stop()
     if args.no_graph:
         launches = csa.launch_count() - n0
     else:
@@ -540,6 +545,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
         e_ends[i].record(stream)
     torch.cuda.synchronize()
     barrier()
+    clk = clocks.stop()
+    if clk is not None and "samples" in clk:
+        clk["window"] = "headline, per-kernel and end-to-end passes"
     e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)) / args.steps
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
 
@@ -598,9 +606,93 @@ def run_gpu(args, cfg, rank, world, local_rank):
         del dc, descs, ws
         torch.cuda.empty_cache()
         line["prefill"] = run_prefill(args, dev, peaks)
+    if world == 1 and not args.no_secondary:
+        line["secondary"] = run_secondary(args, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, seconds_budget=args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def _graph_ms(step, reps, stream):
+    """Median CUDA-event time of a captured step (replayed `reps` times after 3 warm replays)."""
+    import torch
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        step(cap)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    del g
+    return statistics.median(ts)
+
+
+def run_secondary(args, dev, peaks):
+    """The other rows of the path, timed in this run (not the headline):
+    * quant_fp4: the FP4 main-KV encoder over a full 1M-context cache (4 x 2^20
+      rows of fp32 latents -> 288-byte entries), GB/s of its reads + writes;
+    * decode_mx: one decode step of the pages' MXFP4 indexer shape (8 x 65,536
+      positions, 32 heads x 128, top-512), with the MXFP4 scorer's GB/s;
+    * ced_40: one decode step of the 40-layer encoder-decoder stack (4 x
+      131,072 tokens: 2 SWA, 3 x [Full, 5 Reuse] on one entry per 2 tokens,
+      [Full, 3 Reuse] + 4 x [Reindex, 3 Reuse] on the decoder's cache)."""
+    import torch
+    import indexer_selected_sparse_csa2_b200 as csa
+    from csa_synth import get_config
+    from csa_synth.device import DeviceCase
+    stream = torch.cuda.current_stream()
+    out = {}
+    # FP4 encoder
+    n = 4 << 20
+    g = torch.Generator(device=dev).manual_seed(11)
+    src = torch.randn((n, 512), dtype=torch.float32, device=dev, generator=g)
+    dst = torch.empty((n, 288), dtype=torch.uint8, device=dev)
+    ms = _time_ms(lambda: csa.csa_quant_kv(src, csa.CSA_FMT_FP4_E2M1_E4M3X16, dst, stream=stream), 5, stream)
+    nbytes = n * (512 * 4 + 288)
+    out["quant_fp4"] = {"rows": n, "ms": round(ms, 3), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                        "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "bytes": nbytes, "note": "fp32 [4M, 512] read + 288-B entries written"}
+    del src, dst
+    torch.cuda.empty_cache()
+    for name in ("decode_mx", "ced_40"):
+        cfg = get_config(name)
+        dc = DeviceCase(cfg, device=dev)
+        descs = dc.layer_descs(append_rows=True)
+        ws = torch.empty(max(csa.csa_layer_workspace_size(descs), 16), dtype=torch.uint8, device=dev)
+        ms = _graph_ms(lambda st: csa.csa_layer_step(descs, workspace=ws, stream=st), 20, stream)
+        rec = {"workload": name, "B": cfg.B, "T": cfg.T, "H_I": cfg.H_I, "d_I": cfg.d_I, "K": cfg.K,
+               "layers": len(cfg.layers), "ms_per_step": round(ms, 4),
+               "tokens_per_s": round(cfg.B / (ms * 1e-3), 1)}
+        if name == "decode_mx":
+            # the scorer alone (per-kernel events of one captured step)
+            csa.profile_reset()
+            csa.profile_enable(True)
+            csa.csa_layer_step(descs, workspace=ws, stream=stream)
+            torch.cuda.synchronize()
+            csa.profile_enable(False)
+            kern = csa.profile_collect()
+            nl, tot = kern.get("index_score_mx", (0, 0.0))
+            if nl:
+                kb = cfg.B * cfg.T * 68
+                rec["scorer"] = {"kernel": "index_score_mx", "launch_ms": round(tot / nl, 4), "bytes": kb,
+                                 "gbs": round(kb / (tot / nl * 1e-3) / 1e9, 1),
+                                 "hbm_frac": round(kb / (tot / nl * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                 "note": "68 B per key (64 code + 4 exponent bytes); one eager launch with events"}
+        out[name] = rec
+        del dc, descs, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_prefill(args, dev, peaks):
@@ -664,6 +756,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=30.0)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the encoder, decode_mx and ced_40 lines")
     ap.add_argument("--no-graph", action="store_true", help="launch the step eagerly instead of from a CUDA graph")
     ap.add_argument("--flush-l2", action="store_true", help="write 256 MiB between steps even when the step's inputs exceed L2")
     ap.add_argument("--prefill-steps", type=int, default=3)

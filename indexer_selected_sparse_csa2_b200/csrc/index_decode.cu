@@ -298,6 +298,11 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     if (e != cudaSuccess) return e;
   }
   const int64_t nb = a->pool_out ? (a->T + a->pool_block_len - 1) / a->pool_block_len : 0;
+  // a pool-building call whose Top-K is taken inside the pool never reads the
+  // positions' histogram: the scorer skips it
+  const int64_t pool_cap = (int64_t)a->pool_blocks * a->pool_block_len;
+  const bool topk_in_pool = a->pool_out && a->pool_blocks >= a->K && cs_pool_ok(pool_cap);
+  uint32_t* pos_hist = topk_in_pool ? nullptr : w.hist;
   if (a->pool) {
     // pool rows too long for the fused kernel: gathered scoring, then the select
     ScoreParams p{};
@@ -315,9 +320,9 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     p.hist = w.hist;
     e = launch_score_decode(p, B, stream);
   } else if (a->key_format == CSA_KEY_MXFP4) {
-    e = launch_score_mx(a, scores, w.hist, w.bmax, w.bhist, nb, stream);
+    e = launch_score_mx(a, scores, pos_hist, w.bmax, w.bhist, nb, stream);
   } else {
-    e = launch_score_tc(a, scores, w.hist, w.bmax, w.bhist, nb, stream);
+    e = launch_score_tc(a, scores, pos_hist, w.bmax, w.bhist, nb, stream);
   }
   if (e != cudaSuccess) return e;
 
@@ -341,8 +346,7 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     if (e != cudaSuccess) return e;
     if (pool_done && cudaEventRecord(pool_done, stream) != cudaSuccess) return cudaErrorUnknown;
   }
-  const int64_t pool_cap = (int64_t)a->pool_blocks * a->pool_block_len;
-  if (a->pool_out && a->pool_blocks >= a->K && cs_pool_ok(pool_cap)) {
+  if (topk_in_pool) {
     // The K best positions lie in the pool once it keeps >= K blocks: take any
     // of them, p, in block c.  Were c outside the pool, the pool's blocks
     // would all rank above c (larger max, or the same max and a lower block),

@@ -204,7 +204,7 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
       for (int j = 0; j < kMxHeads; ++j) s = fmaf(wj[j], fmaxf(dot[j], 0.f), s);
       if (valid) {
         sc[row] = s;
-        atomicAdd(&h[order_key(s) >> (32 - kHistBits)], 1u);
+        if (p.hist) atomicAdd(&h[order_key(s) >> (32 - kHistBits)], 1u);
       }
       if (build) {
         float m = valid ? s : -INFINITY;
@@ -217,10 +217,10 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
     }
   }
   __syncthreads();
-  uint32_t* gh = p.hist + (int64_t)b * kHistBins;
+  uint32_t* gh = p.hist ? p.hist + (int64_t)b * kHistBins : nullptr;
   uint32_t* gbh = build ? p.bhist + (int64_t)b * kHistBins : nullptr;
   for (int i = tid; i < kHistBins; i += kMxThreads) {
-    if (h[i]) atomicAdd(&gh[i], h[i]);
+    if (gh && h[i]) atomicAdd(&gh[i], h[i]);
     if (build && hb[i]) atomicAdd(&gbh[i], hb[i]);
   }
   if (warp == 1) {

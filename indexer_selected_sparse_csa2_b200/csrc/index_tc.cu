@@ -166,7 +166,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
       const bool valid = row < p.T;
       if (valid) {
         sc[row] = s;
-        atomicAdd(&S.h[order_key(s) >> (32 - kHistBits)], 1u);
+        if (p.hist) atomicAdd(&S.h[order_key(s) >> (32 - kHistBits)], 1u);
       }
       if (build) {
         float m = valid ? s : -INFINITY;
@@ -179,10 +179,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
     }
   }
   __syncthreads();
-  uint32_t* gh = p.hist + (int64_t)b * kHistBins;
+  uint32_t* gh = p.hist ? p.hist + (int64_t)b * kHistBins : nullptr;
   uint32_t* gbh = build ? p.bhist + (int64_t)b * kHistBins : nullptr;
   for (int i = tid; i < kHistBins; i += kTcThreads) {
-    if (S.h[i]) atomicAdd(&gh[i], S.h[i]);
+    if (gh && S.h[i]) atomicAdd(&gh[i], S.h[i]);
     if (build && S.hb[i]) atomicAdd(&gbh[i], S.hb[i]);
   }
   if (warp == 1) {

@@ -22,21 +22,26 @@
 namespace csa {
 
 // ------------------------------------------------------------------ copy --
+constexpr int kCpUnroll = 8;                     // 16-byte loads in flight per thread
+constexpr size_t kCpTile = 256 * kCpUnroll;      // uint4 per CTA tile (32 KB)
+
 __global__ void __launch_bounds__(256) copy_peak_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                                         size_t n16) {
   pdl_enter();
-  const size_t stride = (size_t)gridDim.x * blockDim.x;
-  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  // four independent 16-byte loads in flight per thread
-  for (; i + 3 * stride < n16; i += 4 * stride) {
-    const uint4 a = ld_nc_v4(src + i), b = ld_nc_v4(src + i + stride);
-    const uint4 c = ld_nc_v4(src + i + 2 * stride), d = ld_nc_v4(src + i + 3 * stride);
-    dst[i] = a;
-    dst[i + stride] = b;
-    dst[i + 2 * stride] = c;
-    dst[i + 3 * stride] = d;
+  // contiguous 32 KB tiles, grid-strided; each warp's 8 loads cover 8
+  // consecutive 512-byte segments of its tile
+  const size_t ntiles = n16 / kCpTile;
+  for (size_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    const size_t base = t * kCpTile + threadIdx.x;
+    uint4 v[kCpUnroll];
+#pragma unroll
+    for (int k = 0; k < kCpUnroll; ++k) v[k] = ld_nc_v4(src + base + (size_t)k * 256);
+#pragma unroll
+    for (int k = 0; k < kCpUnroll; ++k) dst[base + (size_t)k * 256] = v[k];
   }
-  for (; i < n16; i += stride) dst[i] = ld_nc_v4(src + i);
+  // ragged tail (< one tile), by the first CTA
+  if (blockIdx.x == 0)
+    for (size_t i = ntiles * kCpTile + threadIdx.x; i < n16; i += blockDim.x) dst[i] = ld_nc_v4(src + i);
 }
 
 // -------------------------------------------------------------- FP8 GEMM --
@@ -211,8 +216,9 @@ csa_status csa_bench_copy(const void* src, void* dst, size_t bytes, csa_stream_t
   if ((bytes & 15) || ((uintptr_t)src & 15) || ((uintptr_t)dst & 15)) return CSA_ERR_ALIGNMENT;
   if (bytes == 0) return CSA_OK;
   const size_t n16 = bytes / 16;
-  size_t g = (n16 + 255) / 256;
+  size_t g = (n16 + kCpTile - 1) / kCpTile;
   const size_t gmax = (size_t)kNumSMs * 8;        // 8 resident CTAs of 256 threads per SM
+  if (g == 0) g = 1;
   if (g > gmax) g = gmax;
   cudaStream_t st = (cudaStream_t)stream;
   {
