@@ -393,6 +393,20 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p
   __shared__ float wgt_s[64];
   __shared__ float inv_s, max_s;
   __shared__ float4 part[kCombGroups - 1][128];
+  const int grp = threadIdx.x >> 7, t = threadIdx.x & 127;
+  const int d = 4 * t;
+  const float* po = p.part_o + ((int64_t)bt * S * H + h) * kD + d;
+  const int64_t sstride = (int64_t)H * kD;
+  // this group's splits grp, grp + 4, ...: the first round of partial loads
+  // (up to 10 per thread) goes out before the merge weights are known, so the
+  // two dependent reads overlap
+  constexpr int kR = 10;
+  uint4 v[kR];
+#pragma unroll
+  for (int k = 0; k < kR; ++k) {
+    const int s = grp + k * kCombGroups;
+    v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
+  }
   const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
   if (threadIdx.x < 32) {
     float M = sk;
@@ -415,31 +429,25 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p
   }
   __syncthreads();
   const float M = max_s;
-  const int grp = threadIdx.x >> 7, t = threadIdx.x & 127;
-  const int d = 4 * t;
   auto weight = [&](int s) -> float {
     if (S <= 64) return wgt_s[s];
     const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
     return m == -INFINITY ? 0.f : exp2f(m - M);
   };
-  const float* po = p.part_o + ((int64_t)bt * S * H + h) * kD + d;
-  const int64_t sstride = (int64_t)H * kD;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  // this group's splits grp, grp + 4, ...: up to 10 loads in flight per round
-  constexpr int kR = 10;
-  for (int s0 = grp; s0 < S; s0 += kR * kCombGroups) {
-    uint4 v[kR];
-#pragma unroll
-    for (int k = 0; k < kR; ++k) {
-      const int s = s0 + k * kCombGroups;
-      v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
-    }
+  for (int s0 = grp;; s0 += kR * kCombGroups) {
 #pragma unroll
     for (int k = 0; k < kR; ++k) {
       const int s = s0 + k * kCombGroups;
       const float w = s < S ? weight(s) : 0.f;
       acc.x += w * __uint_as_float(v[k].x); acc.y += w * __uint_as_float(v[k].y);
       acc.z += w * __uint_as_float(v[k].z); acc.w += w * __uint_as_float(v[k].w);
+    }
+    if (s0 + kR * kCombGroups >= S) break;
+#pragma unroll
+    for (int k = 0; k < kR; ++k) {
+      const int s = s0 + (kR + k) * kCombGroups;
+      v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
     }
   }
   if (grp > 0) part[grp - 1][t] = acc;

@@ -36,7 +36,16 @@
 // Main (FP4) entries are staged as E2M1 * s * 2^-7 (exact in fp16, one
 // multiply per channel pair); their logits are scaled by 2^7 and their
 // probabilities by 2^7 in P, which leaves S and O unchanged.  Window entries
-// are staged unscaled.  All waits are bounded (sm100.cuh).
+// are staged unscaled.
+//
+// With several splits per token the partial O^T (unnormalised) is copied from
+// TMEM into the freed entry-tile buffers as [head][channel] fp32 rows and
+// written to global memory by one 128 KB bulk copy; attn_combine merges the
+// splits.  The kernel triggers its dependents at once and does its prologue
+// (barrier setup, TMEM allocation, the query staging from caller memory or
+// from the stack's staging buffer, which a full event dependency orders)
+// before it waits for the previous kernel on its stream, so the prologue
+// overlaps that kernel's tail.  All waits are bounded (sm100.cuh).
 #include "sm100.cuh"
 #include "q2.cuh"
 #include "attn_tc.cuh"
@@ -73,6 +82,7 @@ struct AtSmem {
   uint8_t* p;       // 2 x (P^T hi, P^T lo)
   float* scl;       // [64] per-head output scale
   float* alpha_s;   // [2][64] by tile parity (a warp may run one tile ahead)
+  int* o_bad;       // O^T not valid (a wait gave up)
   uint64_t* bars;
   uint32_t* tmem_base;
 };
@@ -86,6 +96,7 @@ CSA_DEV AtSmem carve_at(uint8_t* raw) {
   s.p = p; p += 4 * kAtPBytes;
   s.scl = reinterpret_cast<float*>(p); p += 64 * 4;
   s.alpha_s = reinterpret_cast<float*>(p); p += 2 * 64 * 4;
+  s.o_bad = reinterpret_cast<int*>(p); p += 16;
   s.bars = reinterpret_cast<uint64_t*>(p); p += 16 * 8;
   s.tmem_base = reinterpret_cast<uint32_t*>(p);
   return s;
@@ -125,7 +136,7 @@ CSA_DEV bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int code) {
 }
 
 __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcParams p) {
-  pdl_enter();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   AtSmem S = carve_at(smem_raw);
   uint64_t* kv_full = S.bars + 0;    // [2] dequant -> S2 issuer (8 warp arrivals)
@@ -157,6 +168,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     mbar_init(o_done, 1);
     mbar_init(q_full, 1);
     fence_mbar_init();
+    *S.o_bad = 0;
     if (p.q2) {
       // the token's staged query: the tensor-memory part into the (still
       // idle) entry-tile buffers, the shared-memory part straight to its place
@@ -199,7 +211,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   const bool is_deq = warp >= 4 && warp < kAtWarpS;
   // with the query staged by bulk copies the gather warps are free: the first
   // tile's loads go out now, under the staging
-  if (p.q2 && is_deq && nt > 0) CSA_AT_FETCH(tile0);
+  if (p.q2 && is_deq && nt > 0) {
+    pdl_wait();
+    CSA_AT_FETCH(tile0);
+  }
 
   if (warp == kAtWarpS) tmem_alloc(S.tmem_base, kAtTmemCols);
   tc_fence_before();
@@ -298,6 +313,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();                              // the indices and appended rows are ready
 
   if (warp == kAtWarpS) {
     // ------------------------------------------------------------ S2 issuer
@@ -591,20 +607,20 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     // for it), so it could return while that PV still accumulates.
     if (ok && nt > 0) ok = mbar_wait_warp(drain + 1, 0u, kErrWaitAccFull);
     tc_fence_after();
-    for (int c = 0; c < 4; ++c) {
-      // O^T row (position) 128c + 32qtr + lane holds this latent channel
-      const int dp = 128 * c + 32 * qtr + lane;
-      const int d = (dp & ~7) | perm8(dp & 7);
-      // 64 heads of channel d: one 64-column load
-      uint32_t o[64];
-      if (nt > 0 && ok) {
-        tmem_ld64(trow + kAtOCol + 64 * c, o);
-        tmem_wait_ld();
-      } else {
+    if (p.n_splits == 1) {
+      for (int c = 0; c < 4; ++c) {
+        // O^T row (position) 128c + 32qtr + lane holds this latent channel
+        const int dp = 128 * c + 32 * qtr + lane;
+        const int d = (dp & ~7) | perm8(dp & 7);
+        // 64 heads of channel d: one 64-column load
+        uint32_t o[64];
+        if (nt > 0 && ok) {
+          tmem_ld64(trow + kAtOCol + 64 * c, o);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) o[k] = 0u;
-      }
-      if (p.n_splits == 1) {
+          for (int k = 0; k < 64; ++k) o[k] = 0u;
+        }
 #pragma unroll
         for (int hd = 0; hd < kAtH; ++hd) o[hd] = __float_as_uint(__uint_as_float(o[hd]) * S.scl[hd]);
         if (p.rope_cs && c == 3 && qtr >= 2) {
@@ -620,11 +636,45 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
         const int64_t base = (int64_t)bt * kAtH * kD + d;
 #pragma unroll
         for (int hd = 0; hd < kAtH; ++hd) store_out1(p.out, p.out_bf16, base + (int64_t)hd * kD, __uint_as_float(o[hd]));
-      } else {
-        float* dst = p.part_o + ((int64_t)bt * p.n_splits + split) * kAtH * kD + d;
-#pragma unroll
-        for (int hd = 0; hd < kAtH; ++hd) dst[(int64_t)hd * kD] = __uint_as_float(o[hd]);
       }
+    } else if (!ok || nt == 0) {
+      *S.o_bad = 1;
+    }
+  }
+  if (p.n_splits > 1) {
+    // ------------------------------------------------------ partial O^T
+    // the softmax warps have seen the last PV retire; warps w and w + 4 share
+    // TMEM lane quarter w & 3 and copy chunks {0, 1} and {2, 3} into the freed
+    // entry buffers as [head][channel] rows, then one bulk copy writes them
+    __syncthreads();
+    if (warp < 8) {
+      const int qq = warp & 3, cb = 2 * (warp >> 2);
+      const bool valid = *S.o_bad == 0;
+      float* stage = reinterpret_cast<float*>(S.kv);
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = cb + cc;
+        const int dp = 128 * c + 32 * qq + lane;
+        const int d = (dp & ~7) | perm8(dp & 7);
+        uint32_t o[64];
+        if (valid) {
+          tmem_ld64(tbase + ((uint32_t)(32 * qq) << 16) + kAtOCol + 64 * c, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) o[k] = 0u;
+        }
+#pragma unroll
+        for (int hd = 0; hd < kAtH; ++hd) stage[hd * kD + d] = __uint_as_float(o[hd]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store(p.part_o + ((int64_t)bt * p.n_splits + split) * kAtH * kD, S.kv, (uint32_t)(kAtH * kD * 4));
+      bulk_commit();
+      bulk_wait_all();
     }
   }
 #undef CSA_AT_FETCH

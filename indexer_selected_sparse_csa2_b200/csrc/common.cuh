@@ -95,6 +95,12 @@ CSA_DEV void pdl_enter() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+// The two halves, for a kernel whose prologue reads only memory that no
+// kernel of the step writes (caller inputs, or buffers ordered by a full
+// stream-event dependency): it triggers at the top, does that prologue while
+// the previous kernel still runs, and waits before its first other access.
+CSA_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+CSA_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,

@@ -81,6 +81,15 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// Untiled bulk copy this CTA's shared memory -> global (same alignment rules),
+// tracked as a bulk async-group of the issuing thread.
+CSA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+CSA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every bulk async-group of this thread has completed its writes.
+CSA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Untiled bulk copy global -> this CTA's shared memory (no multicast):
 // addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
 CSA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
