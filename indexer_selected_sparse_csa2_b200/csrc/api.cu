@@ -32,7 +32,7 @@ cudaError_t launch_compress(const void* src, int src_dtype, const float* gate, i
                             int64_t dst_row_stride, cudaStream_t stream);
 size_t index_decode_ws_bytes(const csa_index_args* a);
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists,
-                             cudaEvent_t pool_done);
+                             cudaEvent_t pool_done, int64_t safe_rows);
 size_t index_hist_bytes(const csa_index_args* a);
 size_t attn_ws_bytes(const csa_attn_args* a, int share);
 int read_tc_error(bool clear);
@@ -188,7 +188,7 @@ csa_status csa_index_topk(const csa_index_args* a, void* workspace, size_t works
   const size_t need = index_decode_ws_bytes(a);
   if (need > workspace_bytes || (need && !workspace)) return CSA_ERR_WORKSPACE;
   if (!al16(workspace)) return CSA_ERR_ALIGNMENT;
-  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream, nullptr, nullptr));
+  return from_cuda(run_index_decode(a, workspace, (cudaStream_t)stream, nullptr, nullptr, -1));
 }
 
 size_t csa_topk_workspace_size(int32_t B, int64_t n) {
@@ -331,6 +331,43 @@ static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& 
   size_t r = attn_ws_bytes(&at, share);
   if (indexes(L.mode)) r = std::max(r, index_decode_ws_bytes(&ix));
   return al256(r);
+}
+
+// The first key row of `ix` that the stack's prologue (every layer's append
+// jobs) writes, for the full scan that overlaps the prologue: rows below it may
+// be read before the prologue ends.  -1 (wait first) when a job writes the
+// query or the head weights, or when the keys are not a plain E4M3 row cache.
+static int64_t prologue_safe_rows(const csa_layer_desc* layers, int32_t n_layers, const csa_index_args& ix) {
+  if (ix.key_format != CSA_KEY_E4M3 || ix.pool || ix.n_q != 1 || ix.T <= 0) return -1;
+  const int64_t bs = ix.key_batch_stride ? ix.key_batch_stride : ix.key_row_stride * ix.T;
+  const uintptr_t k0 = reinterpret_cast<uintptr_t>(ix.keys);
+  const uintptr_t k1 = k0 + (uintptr_t)((ix.B - 1) * bs + ix.T * ix.key_row_stride);
+  const uintptr_t q0 = reinterpret_cast<uintptr_t>(ix.q), q1 = q0 + (uintptr_t)ix.B * ix.H_I * kDI;
+  const uintptr_t w0 = reinterpret_cast<uintptr_t>(ix.w), w1 = w0 + (uintptr_t)ix.B * ix.H_I * 4;
+  int64_t safe = ix.T;
+  for (int32_t i = 0; i < n_layers; ++i) {
+    for (int k = 0; k < 3; ++k) {
+      const csa_quant_job& q = layers[i].append[k];
+      if (!q.src || q.n_rows <= 0) continue;
+      const int64_t rb = q.fmt == CSA_FMT_FP4_E2M1_E4M3X16 ? kFp4Bytes
+                         : (q.fmt == CSA_FMT_FP8_E4M3_UE8M0X32 ? kFp8Bytes : q.dim);
+      for (int64_t j = 0; j < q.n_rows; ++j) {
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(q.dst) + (uintptr_t)(j * q.dst_row_stride);
+        const uintptr_t a1 = a0 + (uintptr_t)rb;
+        if (a0 < q1 && a1 > q0) return -1;
+        if (a0 < w1 && a1 > w0) return -1;
+        if (a0 >= k1 || a1 <= k0) continue;
+        // the rows this write touches (from its first and last byte)
+        for (uintptr_t a : {a0 < k0 ? k0 : a0, (a1 > k1 ? k1 : a1) - 1}) {
+          const int64_t off = (int64_t)(a - k0);
+          const int64_t t = (off % bs) / ix.key_row_stride;
+          if (t < safe) safe = t;
+        }
+        if (a1 - a0 > (uintptr_t)ix.key_row_stride) safe = 0;   // spans rows: be safe
+      }
+    }
+  }
+  return safe;
 }
 
 static csa_status stack_ws(const csa_layer_desc* layers, int32_t n_layers, StackWs* out) {
@@ -527,7 +564,9 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
           return CSA_ERR_CUDA;
         uint32_t* h = index_hist_bytes(&ix) ? reinterpret_cast<uint32_t*>(hist_base + hist_off) : nullptr;
         hist_off += index_hist_bytes(&ix);
-        if (run_index_decode(&ix, region, ls, h, ix.pool_out ? SS->pool[i] : nullptr) != cudaSuccess) return CSA_ERR_CUDA;
+        if (run_index_decode(&ix, region, ls, h, ix.pool_out ? SS->pool[i] : nullptr,
+                             prologue_safe_rows(layers, n_layers, ix)) != cudaSuccess)
+          return CSA_ERR_CUDA;
       } else if (L.mode == CSA_MODE_REUSE &&
                  cudaStreamWaitEvent(ls, SS->idx[reuse_source(layers, i)], 0) != cudaSuccess) {
         return CSA_ERR_CUDA;

@@ -206,7 +206,7 @@ struct IndexWs {
 static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
-                            int64_t nb, cudaStream_t stream);
+                            int64_t nb, int64_t safe_rows, cudaStream_t stream);
 cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
                             int64_t nb, cudaStream_t stream);
 
@@ -255,9 +255,12 @@ size_t index_hist_bytes(const csa_index_args* a) {
 // without it the workspace's own histograms are cleared here.  `pool_done`:
 // optional event recorded once the candidate pool is written (before the
 // position Top-K of a pool-building call), so that layers searching the pool
-// can start early.
+// can start early.  `safe_rows` (used with `hists` only, i.e. inside a layer
+// stack right after its prologue kernel): key rows below it, and the query and
+// head weights, are not written by that prologue, so the full scan may read
+// them before waiting for it; < 0 waits first.
 cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t stream, uint32_t* hists,
-                             cudaEvent_t pool_done) {
+                             cudaEvent_t pool_done, int64_t safe_rows) {
   if (a->n_q > 1) return run_index_prefill(a, ws, stream);
   IndexWs w = carve_index_ws(a, ws);
   const int B = a->B;
@@ -322,7 +325,7 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
   } else if (a->key_format == CSA_KEY_MXFP4) {
     e = launch_score_mx(a, scores, pos_hist, w.bmax, w.bhist, nb, stream);
   } else {
-    e = launch_score_tc(a, scores, pos_hist, w.bmax, w.bhist, nb, stream);
+    e = launch_score_tc(a, scores, pos_hist, w.bmax, w.bhist, nb, hists ? safe_rows : -1, stream);
   }
   if (e != cudaSuccess) return e;
 

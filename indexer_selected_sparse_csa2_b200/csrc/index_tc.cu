@@ -16,7 +16,12 @@
 //           from TMEM (tcgen05.ld), applies ReLU and the head weights, stores
 //           the fp32 score, adds it to the 4096-bin histogram of the Top-K
 //           select and, when building the candidate pool, the block max.
-// All waits are bounded (see sm100.cuh).
+// Inside a layer stack the scan overlaps the stack's prologue kernel (the
+// appended rows and the cleared histograms): the kernel triggers at once, the
+// producer loads key tiles below `safe_rows` (the first row the prologue
+// writes) before waiting for the prologue, and only the histogram flush and
+// the tiles from safe_rows on wait.  Scores and block maxima go to buffers
+// the prologue does not touch.  All waits are bounded (see sm100.cuh).
 #include "sm100.cuh"
 #include "select.cuh"
 
@@ -45,6 +50,7 @@ struct TcScoreParams {
   uint32_t* bhist;      // [B][4096]
   int64_t nb;
   int block_len;
+  int64_t safe_rows;    // rows below this may be read before the wait; < 0: wait first
 };
 
 struct TcSmem {
@@ -80,7 +86,9 @@ CSA_DEV TcSmem carve_tc_smem(uint8_t* raw) {
 
 __global__ void __launch_bounds__(kTcThreads, 2)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p) {
-  pdl_enter();
+  pdl_trigger();
+  const bool pre = p.safe_rows >= 0;
+  if (!pre) pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   TcSmem S = carve_tc_smem(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -113,9 +121,14 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
 
   if (warp == 0) {
     if (lane == 0) {
+      bool waited = !pre;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % kTcStages;
         const uint32_t ph = (uint32_t)(i / kTcStages) & 1u;
+        if (!waited && (tile0 + i + 1) * kTcRows > p.safe_rows) {
+          pdl_wait();                 // this tile holds rows the prologue writes
+          waited = true;
+        }
         if (!mbar_wait(&S.empty[s], ph ^ 1u, &g_tc_error, kErrWaitSmemEmpty)) break;
         mbar_arrive_expect_tx(&S.full[s], kTcStageBytes);
         tma_load_3d(S.stage + (size_t)s * kTcStageBytes, &tmap, &S.full[s], 0, (int)((tile0 + i) * kTcRows), b);
@@ -179,6 +192,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
     }
   }
   __syncthreads();
+  if (pre) pdl_wait();                    // the histograms were cleared by the prologue
   uint32_t* gh = p.hist ? p.hist + (int64_t)b * kHistBins : nullptr;
   uint32_t* gbh = build ? p.bhist + (int64_t)b * kHistBins : nullptr;
   for (int i = tid; i < kHistBins; i += kTcThreads) {
@@ -224,7 +238,7 @@ bool make_key_tmap(CUtensorMap* map, const uint8_t* keys, int64_t T, int B, int6
 }
 
 cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
-                            int64_t nb, cudaStream_t stream) {
+                            int64_t nb, int64_t safe_rows, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_key_tmap(&map, a->keys, a->T, a->B, a->key_row_stride, a->key_batch_stride))
     return cudaErrorInvalidValue;
@@ -247,6 +261,7 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
   p.bhist = bhist;
   p.nb = nb;
   p.block_len = a->pool_block_len;
+  p.safe_rows = safe_rows;
   static SmemAttrOnce attr;
   const cudaError_t ea = attr.set(index_score_tc_kernel, kTcSmemBytes);
   if (ea != cudaSuccess) return ea;

@@ -257,7 +257,11 @@ __global__ void __launch_bounds__(256) quant_plain_kernel(const void* __restrict
 // are one unit per row; plain casts pack 32 groups of 16 values per unit;
 // the zero range is 512 bytes per unit.
 __global__ void __launch_bounds__(256) quant_batch_kernel(QuantBatch qb) {
-  pdl_enter();
+  // wait, then trigger: a kernel after this one may start before it ends
+  // (the stack's full scan reads the key rows this batch does not write), but
+  // never before the work ahead of this batch on the stream has completed
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t zero_units = (qb.zero_n16 + 31) / 32;
