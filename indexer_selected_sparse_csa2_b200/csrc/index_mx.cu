@@ -11,11 +11,13 @@
 //              into a 4-stage ring;
 //   warp 1     MMA issuer: per tile, one tcgen05.mma kind::f8f6f4 per 32-channel
 //              block (M = 128 keys, N = 32 heads, K = 32) into its own TMEM
-//              accumulator (4 x 32 columns per tile, two tiles in flight);
+//              accumulator (4 x 32 columns per tile, four tiles in flight);
 //   warps 2-5  decode: one key per thread, E2M1 codes -> E4M3 bytes (every
 //              E2M1 value is an E4M3 value) into a 128-byte-swizzled K-major
 //              tile, two tiles in flight;
-//   warps 6-9  epilogue: one key per thread, the 4 x 32 block dots from TMEM,
+//   warps 6-13 epilogue, two groups of four warps taking tiles in turn (one
+//              group alone is latency-bound on its four TMEM round trips per
+//              tile): one key per thread, the 4 x 32 block dots from TMEM,
 //              times 2^e per block, ReLU, head weights, the fp32 score, the
 //              first-level Top-K histogram and, when building the pool, the
 //              block maxima.
@@ -31,9 +33,10 @@ constexpr int kMxStages = 4;
 constexpr int kMxStageBytes = kMxRows * 64;     // packed codes, 8 KB
 constexpr int kMxDec = 2;                       // decoded tiles in flight
 constexpr int kMxDecBytes = kMxRows * 128;      // 16 KB
-constexpr int kMxAcc = 2;
-constexpr uint32_t kMxTmemCols = 256;           // kMxAcc x 4 blocks x 32 heads
-constexpr int kMxThreads = 320;
+constexpr int kMxEpiGroups = 2;
+constexpr int kMxAcc = 2 * kMxEpiGroups;
+constexpr uint32_t kMxTmemCols = 128 * kMxAcc;  // kMxAcc x 4 blocks x 32 heads
+constexpr int kMxThreads = 64 + 128 + 128 * kMxEpiGroups;
 constexpr size_t kMxSmemBytes = 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxDec * kMxDecBytes +
                                 kMxHeads * 128 + 2 * kHistBins * 4 + 256;
 
@@ -168,15 +171,17 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
       if (lane == 0) { mbar_arrive(empty + s); mbar_arrive(dfull + d); }
     }
   } else {
-    // ---- epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31 = keys of the tile
+    // ---- epilogue: group g takes tiles g, g + G, ...; warp w reads TMEM
+    // lanes 32 * (w % 4) .. + 31 = keys of the tile
     const int quarter = warp & 3;
+    const int grp = (warp - 6) >> 2;
     float wj[kMxHeads];
 #pragma unroll
     for (int j = 0; j < kMxHeads; ++j) wj[j] = p.w[(int64_t)b * kMxHeads + j];
     float* sc = p.scores + (int64_t)b * p.T;
     const uint8_t* scb = p.scales + (int64_t)b * p.scale_batch_stride;
     const int bl = p.block_len;
-    for (int i = 0; i < n_my; ++i) {
+    for (int i = grp; i < n_my; i += kMxEpiGroups) {
       const int a = i % kMxAcc;
       const int64_t row = (tile0 + i) * kMxRows + 32 * quarter + lane;
       const bool valid = row < p.T;
@@ -244,7 +249,9 @@ cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hi
   p.scale_batch_stride = a->key_scale_batch_stride;
   p.T = a->T;
   const int64_t ntiles = (a->T + kMxRows - 1) / kMxRows;
-  int64_t ctas_row = (kNumSMs + a->B - 1) / a->B;
+  // one wave: at most one CTA per SM (rounded down, so that no CTA waits
+  // for a second wave)
+  int64_t ctas_row = kNumSMs / a->B;
   if (ctas_row > ntiles) ctas_row = ntiles;
   if (ctas_row < 1) ctas_row = 1;
   p.tiles_per_cta = (int)((ntiles + ctas_row - 1) / ctas_row);

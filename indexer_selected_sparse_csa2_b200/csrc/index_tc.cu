@@ -250,7 +250,7 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
   const int64_t ntiles = (a->T + kTcRows - 1) / kTcRows;
   // two resident CTAs per SM (about 100 KB of shared memory and 128 TMEM
   // columns each): twice the loads in flight and epilogue warps per SM
-  int64_t ctas_row = (2 * kNumSMs + a->B - 1) / a->B;
+  int64_t ctas_row = 2 * kNumSMs / a->B;                 // one wave (rounded down)
   if (ctas_row > ntiles) ctas_row = ntiles;
   if (ctas_row < 1) ctas_row = 1;
   p.tiles_per_cta = (int)((ntiles + ctas_row - 1) / ctas_row);
