@@ -8,7 +8,7 @@
 // where k is the key's E2M1 codes and e its block exponents.
 // Keys sit in two planes: codes [B][T][64 B] and exponent bytes [B][T][4].
 //   warp 0     TMA producer: 128-key x 64-byte code tiles (64-byte swizzle)
-//              into a 4-stage ring;
+//              into a 12-stage ring (96 KB in flight: one CTA per SM);
 //   warp 1     MMA issuer: per tile, one tcgen05.mma kind::f8f6f4 per 32-channel
 //              block (M = 128 keys, N = 32 heads, K = 32) into its own TMEM
 //              accumulator (4 x 32 columns per tile, four tiles in flight);
@@ -29,7 +29,7 @@ namespace csa {
 
 constexpr int kMxRows = 128;                    // keys per tile
 constexpr int kMxHeads = 32;
-constexpr int kMxStages = 4;
+constexpr int kMxStages = 12;                 // 96 KB of key tiles in flight per SM
 constexpr int kMxStageBytes = kMxRows * 64;     // packed codes, 8 KB
 constexpr int kMxDec = 2;                       // decoded tiles in flight
 constexpr int kMxDecBytes = kMxRows * 128;      // 16 KB
@@ -38,7 +38,7 @@ constexpr int kMxAcc = 2 * kMxEpiGroups;
 constexpr uint32_t kMxTmemCols = 128 * kMxAcc;  // kMxAcc x 4 blocks x 32 heads
 constexpr int kMxThreads = 64 + 128 + 128 * kMxEpiGroups;
 constexpr size_t kMxSmemBytes = 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxDec * kMxDecBytes +
-                                kMxHeads * 128 + 2 * kHistBins * 4 + 256;
+                                kMxHeads * 128 + 2 * kHistBins * 4 + 2 * (kMxStages + kMxDec + kMxAcc) * 8 + 16;
 
 static __device__ int g_mx_error;
 
