@@ -219,7 +219,10 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
       float tau[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) tau[k] = (MODE == 1 && k < nlive) ? p.tau[row0 + k] : INFINITY;
-      const float4* wq = reinterpret_cast<const float4*>(S.wts + qg * 64);
+      // the group's 8 x 8 head weights stay in registers for the whole item
+      float2 wr[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) wr[k] = *reinterpret_cast<const float2*>(S.wts + qg * 64 + 2 * k);
       const int kc = (int)(x.kt0 / kPfChunkTiles);
       uint2* cand_base = p.cand + (row0 * p.kchunks + kc) * (int64_t)p.chunk_cap;
       const int nt = (int)n_t;
@@ -245,15 +248,14 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const int k = 4 * hf + kk;
-            const float4 wa = wq[2 * k], wb = wq[2 * k + 1];
             const uint32_t* rr = r32 + 8 * kk;
-            float2 acc = __fmul2_rn(make_float2(wa.x, wa.y), make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
-                                                                        fmaxf(__uint_as_float(rr[1]), 0.f)));
-            acc = __ffma2_rn(make_float2(wa.z, wa.w),
+            float2 acc = __fmul2_rn(wr[4 * k], make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
+                                                           fmaxf(__uint_as_float(rr[1]), 0.f)));
+            acc = __ffma2_rn(wr[4 * k + 1],
                              make_float2(fmaxf(__uint_as_float(rr[2]), 0.f), fmaxf(__uint_as_float(rr[3]), 0.f)), acc);
-            acc = __ffma2_rn(make_float2(wb.x, wb.y),
+            acc = __ffma2_rn(wr[4 * k + 2],
                              make_float2(fmaxf(__uint_as_float(rr[4]), 0.f), fmaxf(__uint_as_float(rr[5]), 0.f)), acc);
-            acc = __ffma2_rn(make_float2(wb.z, wb.w),
+            acc = __ffma2_rn(wr[4 * k + 3],
                              make_float2(fmaxf(__uint_as_float(rr[6]), 0.f), fmaxf(__uint_as_float(rr[7]), 0.f)), acc);
             sc[k] = acc.x + acc.y;
           }
