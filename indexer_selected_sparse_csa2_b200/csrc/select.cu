@@ -420,139 +420,6 @@ __global__ void __launch_bounds__(kFinalThreads, 1) select_final_kernel(SelectJo
   }
 }
 
-// ------------------------------------------------------------ small rows --
-// Rows of at most kSmallCap slots (the Reindex layers' candidate pool): one
-// CTA per row does extract + final in one pass over registers.  Thread t
-// holds slots [16t, 16t + 16); the first-level bin comes from the row's
-// 4096-bin histogram (built by the scorer), and three more radix passes over
-// the keys of that bin (bits 19..12, 11..4, 3..0) give the exact K-th key.
-constexpr int kSmallThreads = 1024;
-constexpr int kSmallPer = kSmallCap / kSmallThreads;
-
-__global__ void __launch_bounds__(kSmallThreads, 1) select_small_kernel(SelectJob J) {
-  pdl_enter();
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x;
-  __shared__ uint32_t warp_tot[32];
-  __shared__ uint32_t total;
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_prefix, s_krem;
-  __shared__ int bin;
-  const int64_t nrow = J.n_row ? min((int64_t)J.n_row[b], J.n) : J.n;
-  const uint32_t K = (uint32_t)J.K;
-  const bool take_all = nrow <= (int64_t)K;
-  // 1. keys of this thread's slots
-  const int s0 = kSmallPer * tid;
-  const float* v = J.vals + (int64_t)b * J.row_stride;
-  uint32_t key[kSmallPer];
-  uint32_t valid = 0;
-#pragma unroll
-  for (int i = 0; i < kSmallPer; i += 4) {
-    float x[4];
-    if (s0 + i + 3 < nrow && ((J.row_stride & 3) == 0) && ((reinterpret_cast<uintptr_t>(J.vals) & 15) == 0)) {
-      const float4 f = *reinterpret_cast<const float4*>(v + s0 + i);
-      x[0] = f.x; x[1] = f.y; x[2] = f.z; x[3] = f.w;
-    } else {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) x[k] = s0 + i + k < nrow ? v[s0 + i + k] : 0.f;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      key[i + k] = order_key(x[k]);
-      if (s0 + i + k < nrow) valid |= 1u << (i + k);
-    }
-  }
-  // 2. exact K-th key tau and the number of keys equal to tau to take
-  if (tid == 0) { s_prefix = 0; s_krem = K; }
-  if (!take_all) {
-    const int beta = threshold_bin<kSmallThreads>(J.hist + (int64_t)b * kHistBins, J.K, warp_tot, &total, &bin);
-    // keys strictly above the first-level bin are all taken
-    uint32_t above = 0;
-#pragma unroll
-    for (int i = 0; i < kSmallPer; ++i)
-      above += ((valid >> i) & 1u) && (int)(key[i] >> (32 - kHistBits)) > beta ? 1u : 0u;
-    block_incl_scan<kSmallThreads>(above, warp_tot, &total);
-    if (tid == 0) { s_prefix = (uint32_t)beta << (32 - kHistBits); s_krem = K - total; }
-    __syncthreads();
-    uint32_t mask = 0xFFFFFFFFu << (32 - kHistBits);
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 12 : (pass == 1 ? 4 : 0);   // bits 19..12, 11..4, 3..0
-      const int width = pass == 2 ? 4 : 8;
-      const uint32_t dmask = (1u << width) - 1u;
-      for (int i = tid; i < 256; i += kSmallThreads) hist[i] = 0;
-      __syncthreads();
-      const uint32_t prefix = s_prefix;
-#pragma unroll
-      for (int i = 0; i < kSmallPer; ++i)
-        if (((valid >> i) & 1u) && (key[i] & mask) == prefix) atomicAdd(&hist[(key[i] >> shift) & dmask], 1u);
-      __syncthreads();
-      if (tid < 32) {
-        // lane l covers digits [255-8l-7, 255-8l], scanning from the top
-        uint32_t loc[8];
-        uint32_t sum = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) { loc[k] = hist[255 - 8 * tid - k]; sum += loc[k]; }
-        uint32_t inc = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
-          if (tid >= o) inc += t;
-        }
-        const uint32_t exc = inc - sum;
-        const uint32_t krem = s_krem;
-        if (exc < krem && inc >= krem) {
-          uint32_t cum = exc;
-          for (int k = 0; k < 8; ++k) {
-            if (cum + loc[k] >= krem) {
-              const uint32_t d = 255u - 8u * tid - k;
-              s_prefix = prefix | (d << shift);
-              s_krem = krem - cum;
-              break;
-            }
-            cum += loc[k];
-          }
-        }
-      }
-      mask |= dmask << shift;
-      __syncthreads();
-    }
-  }
-  __syncthreads();
-  const uint32_t tau = s_prefix;
-  const uint32_t need_eq = s_krem;
-  // 3. ordered emission over this thread's slots
-  uint32_t n_eq = 0;
-  if (!take_all)
-#pragma unroll
-    for (int i = 0; i < kSmallPer; ++i) n_eq += ((valid >> i) & 1u) && key[i] == tau ? 1u : 0u;
-  const uint32_t eq_excl = block_incl_scan<kSmallThreads>(n_eq, warp_tot, &total) - n_eq;
-  uint32_t sel = 0;
-  {
-    uint32_t eq_rank = eq_excl;
-#pragma unroll
-    for (int i = 0; i < kSmallPer; ++i) {
-      bool t = ((valid >> i) & 1u) != 0;
-      if (t && !take_all) {
-        if (key[i] == tau) { t = eq_rank < need_eq; ++eq_rank; }
-        else t = key[i] > tau;
-      }
-      if (t) sel |= 1u << i;
-    }
-  }
-  const uint32_t n_sel = __popc(sel);
-  const uint32_t j0 = block_incl_scan<kSmallThreads>(n_sel, warp_tot, &total) - n_sel;
-  const uint32_t out_count = total;
-  uint32_t j = j0;
-#pragma unroll
-  for (int i = 0; i < kSmallPer; ++i)
-    if ((sel >> i) & 1u) write_selected(J, b, j++, s0 + i);
-  // 4. padding
-  int32_t* out = J.out + (int64_t)b * J.out_stride;
-  for (int64_t jj = (int64_t)out_count * (J.expand ? J.expand : 1) + tid; jj < J.out_width; jj += kSmallThreads)
-    out[jj] = -1;
-}
-
 cudaError_t launch_hist_only(const float* vals, int64_t row_stride, int64_t n, const int32_t* n_row,
                              uint32_t* hist, int B, cudaStream_t stream) {
   SelectJobs js;
@@ -570,15 +437,6 @@ cudaError_t launch_hist_only(const float* vals, int64_t row_stride, int64_t n, c
   dim3 g((p.nchunks + kRunsPerCta - 1) / kRunsPerCta, B, 1);
   ProfScope ps(stream, "select_hist");
   launch_k(select_hist_kernel, dim3(g), dim3(256), 0, stream, js);
-  note_launches(1);
-  return cudaGetLastError();
-}
-
-bool select_small_ok(const SelectJob& j) { return j.n <= kSmallCap && j.expand == 0 && j.hist != nullptr; }
-
-cudaError_t launch_select_small(const SelectJob& j, int B, cudaStream_t stream) {
-  ProfScope ps(stream, "select_small");
-  launch_k(select_small_kernel, dim3(B), dim3(kSmallThreads), 0, stream, j);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -48,12 +48,6 @@ cudaError_t launch_select(const SelectJob* jobs, int njobs, int B, bool build_hi
                           cudaStream_t stream);
 cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t stream);
 
-// Rows of at most kSmallCap slots with a first-level histogram already built
-// and no block expansion: one kernel does the whole select.
-constexpr int kSmallCap = 16384;
-bool select_small_ok(const SelectJob& j);
-cudaError_t launch_select_small(const SelectJob& j, int B, cudaStream_t stream);
-
 // Selection on thread-block clusters (select_cluster.cu): one cluster per
 // (row, job), no workspace beyond the histogram given for rows read from memory.
 struct CsRow {
