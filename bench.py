@@ -412,7 +412,9 @@ def run_gpu(args, cfg, rank, world, local_rank):
     dev = f"cuda:{local_rank}"
     measured_peaks = measure_peaks(dev)
     dc = DeviceCase(cfg, device=dev)
-    descs = dc.layer_descs(append_rows=True)
+    # per-step inputs and outputs packed into one device buffer each (one
+    # host <-> device copy per direction in the end-to-end pass)
+    descs = dc.layer_descs(append_rows=True, packed=True)
     ws_bytes = csa.csa_layer_workspace_size(descs)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
     # L2 between steps: a step that reads more than the L2 holds evicts the
@@ -518,31 +520,49 @@ def run_gpu(args, cfg, rank, world, local_rank):
 
     # ---- end to end through the public call: per-step inputs from pinned host
     # memory, the step, outputs back to pinned host memory
-    h2d_pairs, d2h_pairs = [], []
-    for li, L in enumerate(cfg.layers):
-        dl = dc.layers[li]
-        for tdev in (dl.q, dl.qI, dl.w):
-            h2d_pairs.append((tdev.cpu().pin_memory(), tdev))
-        d2h_pairs.append((torch.empty_like(dl.out, device="cpu").pin_memory(), dl.out))
-        d2h_pairs.append((torch.empty_like(dl.lse, device="cpu").pin_memory(), dl.lse))
-        d2h_pairs.append((torch.empty_like(dl.idx, device="cpu").pin_memory(), dl.idx))
-    for src in dc._append_src:
-        h2d_pairs.append((src.cpu().pin_memory(), src))
-    bi = sum(h.numel() * h.element_size() for h, _ in h2d_pairs)
-    bo = sum(h.numel() * h.element_size() for h, _ in d2h_pairs)
+    # The step's inputs: every layer's attention query (dc.step_q), and its
+    # index queries, head weights and appended source rows (dc.step_in); its
+    # outputs: every layer's out, lse and indices (dc.step_out, layer by
+    # layer).  The small inputs go in on the step's stream before the call;
+    # the queries on a copy stream that the step waits for only before it
+    # first reads them, and each layer's outputs come back on that stream as
+    # soon as the layer is done (csa_layer_step_sync's hooks).
+    h_in = dc.step_in.cpu().pin_memory()
+    h_q = dc.step_q.cpu().pin_memory()
+    h_out = torch.empty_like(dc.step_out, device="cpu").pin_memory()
+    bi = h_in.numel() + h_q.numel()
+    bo = h_out.numel()
+    copy_stream = torch.cuda.Stream()
+    q_ready = torch.cuda.Event()
+    layer_done = [torch.cuda.Event() for _ in cfg.layers]
+    for ev in [q_ready] + layer_done:
+        ev.record(stream)           # (torch creates an event at its first record)
+    torch.cuda.synchronize()
+
+    def step_e2e(i):
+        e_starts[i].record(stream)
+        dc.step_in.copy_(h_in, non_blocking=True)
+        copy_stream.wait_event(e_starts[i])
+        with torch.cuda.stream(copy_stream):
+            dc.step_q.copy_(h_q, non_blocking=True)
+            q_ready.record(copy_stream)
+        # the C-ABI call itself, launched eagerly
+        csa.csa_layer_step(descs, workspace=ws, stream=stream, queries_ready=q_ready, layer_done=layer_done)
+        with torch.cuda.stream(copy_stream):
+            for li, (o0, o1) in enumerate(dc.step_out_ranges):
+                copy_stream.wait_event(layer_done[li])
+                h_out[o0:o1].copy_(dc.step_out[o0:o1], non_blocking=True)
+        stream.wait_stream(copy_stream)
+        e_ends[i].record(stream)
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for _ in range(2):
+        step_e2e(0)                 # warm the eager path (not timed)
     barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush_l2()
-        e_starts[i].record(stream)
-        for h, d in h2d_pairs:
-            d.copy_(h, non_blocking=True)
-        step()                      # the C-ABI call itself, launched eagerly
-        for h, d in d2h_pairs:
-            h.copy_(d, non_blocking=True)
-        e_ends[i].record(stream)
+        step_e2e(i)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
@@ -598,8 +618,11 @@ def run_gpu(args, cfg, rank, world, local_rank):
         "gpu_launches": int(launches),
         "e2e": {"value": round(job_tokens_per_s(cfg.B, world, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo), "ms_per_step": round(e2e_ms, 4),
-                "path": "csa_layer_step called through the Python binding each step (no graph), "
-                        "pinned host inputs copied in and outputs copied back inside the timed events"},
+                "path": "csa_layer_step_sync called through the Python binding each step (no graph); the "
+                        "step's inputs copied in from pinned host memory (index queries, head weights and appended "
+                        "rows before the call; the attention queries on a copy stream the step waits for before "
+                        "it first reads them) and every layer's out, lse and indices copied back to pinned host "
+                        "memory as soon as that layer is done, all inside the timed events"},
         "clocks": clk,
     }
     if world == 1 and not args.no_prefill:

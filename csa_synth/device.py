@@ -117,16 +117,52 @@ class DeviceCase:
         return t.to(torch.bfloat16) if self.cfg.bf16_latents else t
 
     # ------------------------------------------------------------------
-    def layer_descs(self, append_rows: bool = False):
+    def _put(self, arena, t):
+        """Copy ``t`` into the next 256-byte-aligned slot of ``arena`` (a dict
+        holding a uint8 device buffer and a cursor) and return the view."""
+        n = t.numel() * t.element_size()
+        off = (arena["off"] + 255) // 256 * 256
+        if off + n > arena["buf"].numel():
+            raise ValueError("step I/O arena too small")
+        v = arena["buf"][off:off + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        arena["off"] = off + n
+        return v
+
+    def layer_descs(self, append_rows: bool = False, packed: bool = False):
         """ctypes LayerDesc array for the config's stack.  With ``append_rows``
         every owner layer re-encodes the newest token (position T-1) of its
         main KV and indexer key, and every layer its newest window row, as part
-        of the step (values from the seeded generator)."""
+        of the step (values from the seeded generator).  With ``packed`` the
+        step's per-token inputs are moved into two contiguous device buffers,
+        ``self.step_q`` (every layer's attention query) and ``self.step_in``
+        (index queries, head weights, appended source rows), and its outputs
+        (out, lse, idx of every layer, layer by layer) into ``self.step_out``
+        with layer i at bytes ``self.step_out_ranges[i]``, so that a caller
+        moves each with one host <-> device copy (per layer for the outputs)."""
         import torch
         csa = _lib()
         cfg = self.cfg
         descs = []
         self._append_src = []
+        src_arena = None
+        if packed:
+            per_tok = 4 * (2 * 512 + cfg.d_I) * max(cfg.n_q, 1)
+            n_in = sum(dl.q.numel() * 4 + dl.qI.numel() + dl.w.numel() * 4 + 1024 for dl in self.layers)
+            n_in += len(cfg.layers) * (cfg.B * per_tok + 1024)
+            src_arena = {"buf": torch.empty(n_in, dtype=torch.uint8, device=self.device), "off": 0}
+            n_q = sum(dl.q.numel() * 4 + 256 for dl in self.layers)
+            q_arena = {"buf": torch.empty(n_q, dtype=torch.uint8, device=self.device), "off": 0}
+            n_out = sum(dl.out.numel() * 4 + dl.lse.numel() * 4 + dl.idx.numel() * 4 + 1024 for dl in self.layers)
+            out_arena = {"buf": torch.empty(n_out, dtype=torch.uint8, device=self.device), "off": 0}
+            self.step_out_ranges = []
+            for dl in self.layers:
+                dl.q = self._put(q_arena, dl.q)
+                dl.qI, dl.w = (self._put(src_arena, t) for t in (dl.qI, dl.w))
+                o0 = (out_arena["off"] + 255) // 256 * 256
+                dl.out, dl.lse, dl.idx = (self._put(out_arena, t) for t in (dl.out, dl.lse, dl.idx))
+                self.step_out_ranges.append((o0, out_arena["off"]))
+        put = (lambda t: self._put(src_arena, t)) if packed else (lambda t: t)
         for li, L in enumerate(cfg.layers):
             d = csa.LayerDesc()
             d.mode = L.mode
@@ -158,6 +194,9 @@ class DeviceCase:
                         kx = torch.from_numpy(wl.index_key(cfg, o, 0, t_new, n_new)).to(self.device)
                         kvrow, krow = self.kv[o][0, t_new:], self.keys[o][0, t_new:]
                         kv_stride, k_stride = self.kv[o].stride(1), self.keys[o].stride(1)
+                    mx = put(mx)
+                    if cfg.key_format == "e4m3":
+                        kx = put(kx)
                     jobs.append(csa.quant_job(mx, csa.CSA_FMT_FP4_E2M1_E4M3X16, kvrow, kv_stride))
                     if cfg.key_format == "e4m3":       # (MXFP4 keys are encoded whole above)
                         jobs.append(csa.quant_job(kx, csa.CSA_FMT_FP8_E4M3_PLAIN, krow, k_stride))
@@ -170,6 +209,7 @@ class DeviceCase:
                 else:
                     wx = self._latent_tensor(wl.window_latent(cfg, li, 0)[r0:])
                     wrow, w_stride = dl.win[0, r0:], dl.win.stride(1)
+                wx = put(wx)
                 jobs.append(csa.quant_job(wx, csa.CSA_FMT_FP8_E4M3_UE8M0X32, wrow, w_stride))
                 self._append_src.append(wx)
                 for k, j in enumerate(jobs):
@@ -185,4 +225,8 @@ class DeviceCase:
                                    sink=dl.sink, K=0)
             d._keep = (getattr(d, "_keep", None), self.keys, self.kv, dl)
             descs.append(d)
+        if packed:
+            self.step_in = src_arena["buf"][:src_arena["off"]]
+            self.step_q = q_arena["buf"][:q_arena["off"]]
+            self.step_out = out_arena["buf"][:out_arena["off"]]
         return csa.make_layer_array(descs)

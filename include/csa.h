@@ -298,6 +298,26 @@ size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers);
 csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
                           size_t workspace_bytes, csa_stream_t stream);
 
+/* csa_layer_step with hooks for overlapping host <-> device transfers with
+ * the step (no counterpart on the pages; a serving loop's copies).  Every
+ * field may be NULL; events are cudaEvent_t of the stream's device.
+ *   queries_ready : the step reads the layers' attention queries (attn.q)
+ *                   only after this event completes, so their upload may
+ *                   still be in flight on another stream when the call is
+ *                   made.  Everything else (appended rows, index queries and
+ *                   weights, caches) must be ready as for csa_layer_step.
+ *   layer_done[i] : recorded once layer i's outputs (attn.out, attn.lse and,
+ *                   for an indexing layer, index.idx) are written, so that
+ *                   their download can start while later layers still run.
+ * Ordering on `stream` is as for csa_layer_step (the call's end on `stream`
+ * follows every layer). */
+typedef struct {
+  void* queries_ready;
+  void* layer_done[64];
+} csa_step_sync;
+csa_status csa_layer_step_sync(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
+                               size_t workspace_bytes, const csa_step_sync* sync, csa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Opt-in timing of the library's own kernels (profiling support, no
  * counterpart on the pages).  While enabled, each kernel launch is bracketed

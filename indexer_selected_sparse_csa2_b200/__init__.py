@@ -97,6 +97,14 @@ _attn_ws = _sig("csa_attn_workspace_size", ctypes.c_size_t, [ctypes.POINTER(Attn
 _attn = _sig("csa_sparse_attn", _i32, [ctypes.POINTER(AttnArgs), _p, ctypes.c_size_t, _p])
 _layer_ws = _sig("csa_layer_workspace_size", ctypes.c_size_t, [ctypes.POINTER(LayerDesc), _i32])
 _layer = _sig("csa_layer_step", _i32, [ctypes.POINTER(LayerDesc), _i32, _p, ctypes.c_size_t, _p])
+
+
+class StepSync(ctypes.Structure):
+    _fields_ = [("queries_ready", _p), ("layer_done", _p * 64)]
+
+
+_layer_sync = _sig("csa_layer_step_sync", _i32,
+                   [ctypes.POINTER(LayerDesc), _i32, _p, ctypes.c_size_t, ctypes.POINTER(StepSync), _p])
 _status_string = _sig("csa_status_string", ctypes.c_char_p, [_i32])
 _launch_count = _sig("csa_launch_count", ctypes.c_uint64, [])
 _device_status = _sig("csa_device_status", _i32, [])
@@ -119,7 +127,7 @@ EXPORTED = ["csa_quant_kv", "csa_compress_kv", "csa_quant_mxfp4", "csa_index_wor
             "csa_profile_enable", "csa_profile_collect", "csa_index_topk_noalloc", "csa_device_status",
             "csa_index_noalloc_capacity", "csa_profile_snapshot", "csa_profile_reset",
             "csa_bench_copy", "csa_bench_fp8_gemm", "csa_cp_local_pairs", "csa_cp_merge_workspace_size",
-            "csa_cp_merge_topk", "csa_cp_localize", "csa_cp_combine"]
+            "csa_cp_merge_topk", "csa_cp_localize", "csa_cp_combine", "csa_layer_step_sync"]
 
 
 def profile_enable(on: bool) -> bool:
@@ -301,13 +309,31 @@ def csa_layer_workspace_size(layers) -> int:
     return int(_layer_ws(layers, len(layers)))
 
 
-def csa_layer_step(layers, workspace=None, stream=None, device=None) -> None:
-    """Run a ctypes array of LayerDesc (see ``make_layer_array``) on one stream."""
+def _event(ev) -> Optional[int]:
+    if ev is None:
+        return None
+    return ev.cuda_event if hasattr(ev, "cuda_event") else int(ev)
+
+
+def csa_layer_step(layers, workspace=None, stream=None, device=None, queries_ready=None, layer_done=None) -> None:
+    """Run a ctypes array of LayerDesc (see ``make_layer_array``) on one stream.
+    ``queries_ready`` (a torch.cuda.Event) and ``layer_done`` (one event or
+    None per layer) select csa_layer_step_sync: the step reads the attention
+    queries only after ``queries_ready`` and records ``layer_done[i]`` once
+    layer i's outputs are written."""
     # the library checks a given workspace's size itself; query it only to allocate one
     if workspace is None:
         workspace = _workspace(csa_layer_workspace_size(layers), device or "cuda")
     nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(_layer(layers, len(layers), _ptr(workspace), nbytes, _stream(stream)), "csa_layer_step")
+    if queries_ready is None and layer_done is None:
+        _check(_layer(layers, len(layers), _ptr(workspace), nbytes, _stream(stream)), "csa_layer_step")
+        return
+    sync = StepSync()
+    sync.queries_ready = _event(queries_ready)
+    for i, ev in enumerate(layer_done or []):
+        sync.layer_done[i] = _event(ev)
+    _check(_layer_sync(layers, len(layers), _ptr(workspace), nbytes, ctypes.byref(sync), _stream(stream)),
+           "csa_layer_step_sync")
 
 
 def csa_bench_copy(src, dst, stream=None) -> None:

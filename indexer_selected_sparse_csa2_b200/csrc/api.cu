@@ -415,6 +415,7 @@ size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) 
 // capture the fork / join below becomes graph edges.
 constexpr int kAuxStreams = 8;
 constexpr int kMaxStackLayers = 64;
+static_assert(sizeof(csa_step_sync::layer_done) / sizeof(void*) == kMaxStackLayers, "csa_step_sync layout");
 struct StackStreams {
   cudaStream_t aux[kAuxStreams] = {};
   cudaEvent_t start = nullptr;   // the caller's stream at the start of a step
@@ -454,6 +455,11 @@ static StackStreams* stack_streams() {
 
 csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
                           size_t workspace_bytes, csa_stream_t stream) {
+  return csa_layer_step_sync(layers, n_layers, workspace, workspace_bytes, nullptr, stream);
+}
+
+csa_status csa_layer_step_sync(const csa_layer_desc* layers, int32_t n_layers, void* workspace,
+                               size_t workspace_bytes, const csa_step_sync* sync, csa_stream_t stream) {
   if (!layers || n_layers < 1) return CSA_ERR_INVALID_ARG;
   if (n_layers > kMaxStackLayers) return CSA_ERR_UNSUPPORTED;
   // validate everything before enqueuing anything
@@ -510,10 +516,13 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       return true;
     };
     const bool staged = w.q2 > 0;
+    cudaEvent_t q_ready = sync ? static_cast<cudaEvent_t>(sync->queries_ready) : nullptr;
     if (staged) {
       used[kAuxStreams - 1] = true;
       if (cudaEventRecord(SS->start, st) != cudaSuccess || cudaStreamWaitEvent(sst, SS->start, 0) != cudaSuccess)
         return CSA_ERR_CUDA;
+      // the staging is the first reader of the attention queries
+      if (q_ready && cudaStreamWaitEvent(sst, q_ready, 0) != cudaSuccess) return CSA_ERR_CUDA;
     }
     size_t q2_off = 0;
     for (int32_t i = 0; i < n_layers; ++i) {
@@ -575,7 +584,10 @@ csa_status csa_layer_step(const csa_layer_desc* layers, int32_t n_layers, void* 
       const void* q2 = layer_q2_bytes(at) ? q2_base + q2_off : nullptr;
       q2_off += layer_q2_bytes(at);
       if (q2 && cudaStreamWaitEvent(ls, SS->stg, 0) != cudaSuccess) return CSA_ERR_CUDA;
+      if (!q2 && q_ready && cudaStreamWaitEvent(ls, q_ready, 0) != cudaSuccess) return CSA_ERR_CUDA;
       if (run_sparse_attn(&at, region, ls, q2, share) != cudaSuccess) return CSA_ERR_CUDA;
+      if (sync && sync->layer_done[i] && cudaEventRecord(static_cast<cudaEvent_t>(sync->layer_done[i]), ls) != cudaSuccess)
+        return CSA_ERR_CUDA;
     }
     return CSA_OK;
   };

@@ -129,3 +129,47 @@ def test_cold_step_body(csa):
         pytest.skip("runs in a fresh process under test_cold_first_step")
     for fill in (0, 255):
         _check_stack(csa, get_config("decode_64k", B=8, T=20000), append=True, ws_fill=fill)
+
+
+def test_step_sync_hooks_match_plain_step(csa):
+    """csa_layer_step_sync: the attention queries uploaded on another stream
+    behind a long copy, the step told to wait for them, and every layer's
+    outputs downloaded as soon as its layer_done event fires, give the same
+    bytes as csa_layer_step with everything resident (4-layer pool stack with
+    appends, packed step I/O)."""
+    from csa_synth.device import DeviceCase
+    cfg = get_config("hier_1m", B=2, T=1 << 15)
+    dc = DeviceCase(cfg)
+    descs = dc.layer_descs(append_rows=True, packed=True)
+    ws = torch.empty(csa.csa_layer_workspace_size(descs), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    csa.csa_layer_step(descs, workspace=ws, stream=stream)
+    torch.cuda.synchronize()
+    want = dc.step_out.cpu().clone()
+    h_q = dc.step_q.cpu().pin_memory()
+    h_out = torch.zeros_like(dc.step_out, device="cpu").pin_memory()
+    # the queries are destroyed on the device and come back only through the
+    # copy stream, after a 256 MiB device copy that delays them
+    dc.step_q.zero_()
+    dc.step_out.zero_()
+    big_a = torch.empty(1 << 28, dtype=torch.uint8, device="cuda")
+    big_b = torch.empty_like(big_a)
+    torch.cuda.synchronize()
+    copy_stream = torch.cuda.Stream()
+    q_ready = torch.cuda.Event()
+    done = [torch.cuda.Event() for _ in cfg.layers]
+    for ev in [q_ready] + done:
+        ev.record(stream)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(copy_stream):
+        big_b.copy_(big_a)
+        dc.step_q.copy_(h_q, non_blocking=True)
+        q_ready.record(copy_stream)
+    csa.csa_layer_step(descs, workspace=ws, stream=stream, queries_ready=q_ready, layer_done=done)
+    with torch.cuda.stream(copy_stream):
+        for li, (o0, o1) in enumerate(dc.step_out_ranges):
+            copy_stream.wait_event(done[li])
+            h_out[o0:o1].copy_(dc.step_out[o0:o1], non_blocking=True)
+    torch.cuda.synchronize()
+    for li, (o0, o1) in enumerate(dc.step_out_ranges):
+        assert torch.equal(h_out[o0:o1], want[o0:o1]), f"layer {li}"
