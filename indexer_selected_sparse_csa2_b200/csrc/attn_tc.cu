@@ -674,7 +674,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     if (tid == 0) {
       bulk_store(p.part_o + ((int64_t)bt * p.n_splits + split) * kAtH * kD, S.kv, (uint32_t)(kAtH * kD * 4));
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();                    // the CTA's shared memory must outlive the copy's reads
     }
   }
 #undef CSA_AT_FETCH

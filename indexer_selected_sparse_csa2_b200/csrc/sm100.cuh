@@ -88,8 +88,10 @@ CSA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
                ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
 }
 CSA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until every bulk async-group of this thread has completed its writes.
-CSA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until every bulk async-group of this thread has read its source (the
+// shared memory may then be reused or released); the writes themselves are
+// visible to work ordered after the kernel, as any store of the kernel is.
+CSA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Untiled bulk copy global -> this CTA's shared memory (no multicast):
 // addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
 CSA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
