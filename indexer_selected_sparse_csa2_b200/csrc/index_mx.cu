@@ -12,12 +12,10 @@
 //   warp 1     MMA issuer: per tile, one tcgen05.mma kind::f8f6f4 per 32-channel
 //              block (M = 128 keys, N = 32 heads, K = 32) into its own TMEM
 //              accumulator (4 x 32 columns per tile, four tiles in flight);
-//   warps 2-5  decode: one key per thread, E2M1 codes -> E4M3 bytes (every
-//              E2M1 value is an E4M3 value) into a 128-byte-swizzled K-major
-//              tile, two tiles in flight;
-//   warps 6-13 epilogue, two groups of four warps taking tiles in turn (one
-//              group alone is latency-bound on its four TMEM round trips per
-//              tile): one key per thread, the 4 x 32 block dots from TMEM,
+//   warps 2-9  decode: two threads per key (64 channels each), E2M1 codes ->
+//              E4M3 bytes (every E2M1 value is an E4M3 value) into a
+//              128-byte-swizzled K-major tile, four tiles in flight;
+//   warps 10-13 epilogue: one key per thread, the 4 x 32 block dots from TMEM,
 //              times 2^e per block, ReLU, head weights, the fp32 score, the
 //              first-level Top-K histogram and, when building the pool, the
 //              block maxima.
@@ -31,12 +29,14 @@ constexpr int kMxRows = 128;                    // keys per tile
 constexpr int kMxHeads = 32;
 constexpr int kMxStages = 12;                 // 96 KB of key tiles in flight per SM
 constexpr int kMxStageBytes = kMxRows * 64;     // packed codes, 8 KB
-constexpr int kMxDec = 2;                       // decoded tiles in flight
+constexpr int kMxDec = 4;                       // decoded tiles in flight
+constexpr int kMxDecWarps = 8;
 constexpr int kMxDecBytes = kMxRows * 128;      // 16 KB
-constexpr int kMxEpiGroups = 2;
-constexpr int kMxAcc = 2 * kMxEpiGroups;
+constexpr int kMxEpiGroups = 1;
+constexpr int kMxAcc = 4;
 constexpr uint32_t kMxTmemCols = 128 * kMxAcc;  // kMxAcc x 4 blocks x 32 heads
-constexpr int kMxThreads = 64 + 128 + 128 * kMxEpiGroups;
+constexpr int kMxEpiWarp0 = 2 + kMxDecWarps;
+constexpr int kMxThreads = 32 * kMxEpiWarp0 + 128 * kMxEpiGroups;
 constexpr size_t kMxSmemBytes = 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxDec * kMxDecBytes +
                                 kMxHeads * 128 + 2 * kHistBins * 4 + 2 * (kMxStages + kMxDec + kMxAcc) * 8 + 16;
 
@@ -94,8 +94,8 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
   const bool build = p.bmax != nullptr;
 
   if (tid == 0) {
-    for (int i = 0; i < kMxStages; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 4); }
-    for (int i = 0; i < kMxDec; ++i) { mbar_init(dfull + i, 4); mbar_init(dempty + i, 1); }
+    for (int i = 0; i < kMxStages; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, kMxDecWarps); }
+    for (int i = 0; i < kMxDec; ++i) { mbar_init(dfull + i, kMxDecWarps); mbar_init(dempty + i, 1); }
     for (int i = 0; i < kMxAcc; ++i) { mbar_init(accf + i, 1); mbar_init(acce + i, 4); }
     fence_mbar_init();
     prefetch_tmap(&tmap);
@@ -141,9 +141,10 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
         mma_commit(accf + a);
       }
     }
-  } else if (warp < 6) {
-    // ---- decode: thread = key row r of the tile
-    const int r = tid - 64;
+  } else if (warp < kMxEpiWarp0) {
+    // ---- decode: threads 2r and 2r + 1 take key row r, packed chunks
+    // {0, 1} and {2, 3} (64 channels each)
+    const int r = (tid - 64) >> 1, hf = (tid - 64) & 1;
     for (int i = 0; i < n_my; ++i) {
       const int s = i % kMxStages, d = i % kMxDec;
       bool ok = __all_sync(0xffffffffu, mbar_wait(full + s, (uint32_t)(i / kMxStages) & 1u, &g_mx_error, kErrWaitTmaFull));
@@ -154,7 +155,8 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
       const uint8_t* src = stage + (size_t)s * kMxStageBytes + r * 64;
       uint8_t* dst = dec + (size_t)d * kMxDecBytes + r * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * hf + cc;
         // packed chunk c (channels 32c .. 32c + 31) at its 64-byte-swizzle position
         const uint4 v = *reinterpret_cast<const uint4*>(src + ((c ^ ((r >> 1) & 3)) << 4));
         const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -174,18 +176,26 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
     // ---- epilogue: group g takes tiles g, g + G, ...; warp w reads TMEM
     // lanes 32 * (w % 4) .. + 31 = keys of the tile
     const int quarter = warp & 3;
-    const int grp = (warp - 6) >> 2;
+    const int grp = (warp - kMxEpiWarp0) >> 2;
     float wj[kMxHeads];
 #pragma unroll
     for (int j = 0; j < kMxHeads; ++j) wj[j] = p.w[(int64_t)b * kMxHeads + j];
     float* sc = p.scores + (int64_t)b * p.T;
     const uint8_t* scb = p.scales + (int64_t)b * p.scale_batch_stride;
     const int bl = p.block_len;
+    // exponent bytes of this lane's key, loaded one tile of this group ahead
+    // (a load at the top of each tile would expose its latency every tile)
+    auto exps = [&](int i) -> uint32_t {
+      const int64_t r = (tile0 + i) * kMxRows + 32 * quarter + lane;
+      return (i < n_my && r < p.T) ? *reinterpret_cast<const uint32_t*>(scb + r * p.scale_row_stride) : 0x7F7F7F7Fu;
+    };
+    uint32_t e_next = exps(grp);
     for (int i = grp; i < n_my; i += kMxEpiGroups) {
       const int a = i % kMxAcc;
       const int64_t row = (tile0 + i) * kMxRows + 32 * quarter + lane;
       const bool valid = row < p.T;
-      const uint32_t ebytes = valid ? *reinterpret_cast<const uint32_t*>(scb + row * p.scale_row_stride) : 0x7F7F7F7Fu;
+      const uint32_t ebytes = e_next;
+      e_next = exps(i + kMxEpiGroups);
       if (!__all_sync(0xffffffffu, mbar_wait(accf + a, (uint32_t)(i / kMxAcc) & 1u, &g_mx_error, kErrWaitAccFull))) break;
       tc_fence_after();
       float dot[kMxHeads];
