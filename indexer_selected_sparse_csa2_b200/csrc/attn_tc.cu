@@ -22,8 +22,10 @@
 // Warp roles: warps 0-3 softmax / output (one TMEM lane quarter each; the
 // two lanes of a head split the tile's entries), warps 4-11 gather +
 // dequantise (8 lanes take 8 entries, 4 lanes per entry, 128 channels each;
-// the next tile's raw bytes are loaded into registers while the current one
-// is decoded), warp 12 issues the S2 MMAs, warp 13 the PV MMAs.  Entry
+// the codes of the next tile's entries are staged by cp.async into each
+// lane's own 128-byte shared-memory slot, and their block scales loaded,
+// while the current tile is decoded), warp 12 issues the S2 MMAs, warp 13 the
+// PV MMAs.  Entry
 // tiles and P are double buffered, so tile i+1 is dequantised while S2, the
 // softmax and PV of tile i run.  Online softmax in the exp2 domain with lazy
 // rescaling: the running max only moves when a tile's max exceeds it by more
@@ -65,7 +67,9 @@ constexpr int kAtQBlkBytes = 128 * 128;             // 128 rows x 64 fp16
 constexpr int kAtKVBlk = kAtE * 128;                // one 64-channel block of an entry tile
 constexpr int kAtKVBytes = 8 * kAtKVBlk;            // 64 KB
 constexpr int kAtPBytes = kAtH * kAtE * 2;          // P^T part (hi or lo): 64 head rows x 128 B
-constexpr size_t kAtSmemBytes = 1024 + (size_t)kAtQSmemBlocks * kAtQBlkBytes + 2 * kAtKVBytes + 4 * kAtPBytes + 1024;
+constexpr int kAtRawBytes = 256 * 128;            // cp.async staging: one 128-byte slot per gather thread
+constexpr size_t kAtSmemBytes =
+    1024 + (size_t)kAtQSmemBlocks * kAtQBlkBytes + 2 * kAtKVBytes + 4 * kAtPBytes + kAtRawBytes + 1024;
 constexpr uint32_t kAtTmemCols = 512;
 constexpr uint32_t kAtSCol = 32 * kAtQTmemBlocks;   // S2: 64 fp32 columns after Q2
 constexpr uint32_t kAtOCol = 256;                   // O^T chunk c: columns 256 + 64c
@@ -80,6 +84,7 @@ struct AtSmem {
   uint8_t* q2;      // Q2 channels 384..511 (2 blocks)
   uint8_t* kv;      // 2 entry tiles
   uint8_t* p;       // 2 x (P^T hi, P^T lo)
+  uint8_t* raw;     // [256 gather threads][128 B] staged entry codes
   float* scl;       // [64] per-head output scale
   float* alpha_s;   // [2][64] by tile parity (a warp may run one tile ahead)
   int* o_bad;       // O^T not valid (a wait gave up)
@@ -94,6 +99,7 @@ CSA_DEV AtSmem carve_at(uint8_t* raw) {
   s.q2 = p; p += kAtQSmemBlocks * kAtQBlkBytes;
   s.kv = p; p += 2 * kAtKVBytes;
   s.p = p; p += 4 * kAtPBytes;
+  s.raw = p; p += kAtRawBytes;
   s.scl = reinterpret_cast<float*>(p); p += 64 * 4;
   s.alpha_s = reinterpret_cast<float*>(p); p += 2 * 64 * 4;
   s.o_bad = reinterpret_cast<int*>(p); p += 16;
@@ -186,27 +192,31 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   const int32_t* idx_b = p.idx + (int64_t)bt * p.K;
   const uint8_t* kvb = p.kv + (int64_t)b * p.kv_batch_stride;
   const uint8_t* wb = p.win ? p.win + (int64_t)b * p.win_batch_stride : nullptr;
-  uint4 rr[8];
   uint2 rex = make_uint2(0, 0);
   int kind = 0;   // 0 invalid, 1 FP4 main entry, 2 FP8 window entry
-#define CSA_AT_FETCH(tile)                                                                     \
-  do {                                                                                         \
-    const int jj = (tile) * kAtE + e;                                                          \
-    kind = 0;                                                                                  \
-    if (jj < p.K) {                                                                            \
-      const int pos = idx_b[jj];                                                               \
-      if (pos >= 0) {                                                                          \
-        const uint8_t* row = kvb + (int64_t)pos * p.kv_row_stride;                             \
-        _Pragma("unroll") for (int k = 0; k < 4; ++k) rr[k] = ld_nc_v4(row + 64 * q4 + 16 * k); \
-        rex = *reinterpret_cast<const uint2*>(row + 256 + 8 * q4);                             \
-        kind = 1;                                                                              \
-      }                                                                                        \
-    } else if (jj < p.n_entries) {                                                             \
-      const uint8_t* row = wb + (int64_t)(tq + jj - p.K) * p.win_row_stride;                   \
-      _Pragma("unroll") for (int k = 0; k < 8; ++k) rr[k] = ld_nc_v4(row + 128 * q4 + 16 * k); \
-      rex.x = *reinterpret_cast<const uint32_t*>(row + 512 + 4 * q4);                          \
-      kind = 2;                                                                                \
-    }                                                                                          \
+  // this lane's staging slot; chunk k sits at chunk k ^ (jd & 7), so the
+  // 8-lane groups of a warp read different banks
+  const int swz = jd & 7;
+  const uint32_t slot = smem_u32(S.raw) + 128u * (uint32_t)(jd & 255);
+#define CSA_AT_FETCH(tile)                                                                                 \
+  do {                                                                                                     \
+    const int jj = (tile) * kAtE + e;                                                                      \
+    kind = 0;                                                                                              \
+    if (jj < p.K) {                                                                                        \
+      const int pos = idx_b[jj];                                                                           \
+      if (pos >= 0) {                                                                                      \
+        const uint8_t* row = kvb + (int64_t)pos * p.kv_row_stride;                                         \
+        _Pragma("unroll") for (int k = 0; k < 4; ++k) cp_async16(slot + 16u * (k ^ swz), row + 64 * q4 + 16 * k); \
+        rex = *reinterpret_cast<const uint2*>(row + 256 + 8 * q4);                                         \
+        kind = 1;                                                                                          \
+      }                                                                                                    \
+    } else if (jj < p.n_entries) {                                                                         \
+      const uint8_t* row = wb + (int64_t)(tq + jj - p.K) * p.win_row_stride;                               \
+      _Pragma("unroll") for (int k = 0; k < 8; ++k) cp_async16(slot + 16u * (k ^ swz), row + 128 * q4 + 16 * k); \
+      rex.x = *reinterpret_cast<const uint32_t*>(row + 512 + 4 * q4);                                      \
+      kind = 2;                                                                                            \
+    }                                                                                                      \
+    cp_async_commit();                                                                                     \
   } while (0)
   const bool is_deq = warp >= 4 && warp < kAtWarpS;
   // with the query staged by bulk copies the gather warps are free: the first
@@ -379,6 +389,15 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       const int bi = i & 1;
       if (i >= 2 && !mbar_wait_warp(kv_free + bi, (uint32_t)((i >> 1) - 1) & 1u, kErrWaitSmemEmpty)) break;
       uint8_t* kt = S.kv + bi * kAtKVBytes;
+      // this lane's staged codes (its own cp.async copies: no barrier needed)
+      cp_async_wait_all();
+      uint4 rr[8];
+      {
+        const uint8_t* rs = S.raw + 128 * (jd & 255);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          rr[k] = (k < 4 || kind == 2) ? *reinterpret_cast<const uint4*>(rs + 16 * (k ^ swz)) : make_uint4(0, 0, 0, 0);
+      }
       // channels [128*q4, 128*q4 + 128) of entry e, one 16-byte chunk (8
       // positions) per group of 8 channels
       if (kind == 1) {
@@ -442,6 +461,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       if (lane == 0) mbar_arrive(kv_full + bi);
       if (i + 1 < nt) CSA_AT_FETCH(tile0 + i + 1);
     }
+    cp_async_wait_all();    // none in flight when the CTA leaves (also after an early break)
   } else {
     // ---------------------------------------------------------------- softmax
     const int qtr = warp;                      // TMEM lanes 32*qtr .. +31

@@ -81,6 +81,14 @@ CSA_DEV void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int c
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
 }
+// 16-byte asynchronous copy global -> shared (cp.async, L2 only), 16-byte
+// aligned on both sides; the issuing thread waits for its own copies with
+// cp_async_wait_all() before it reads the destination.
+CSA_DEV void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 // Untiled bulk copy this CTA's shared memory -> global (same alignment rules),
 // tracked as a bulk async-group of the issuing thread.
 CSA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
