@@ -22,6 +22,8 @@
 //      so S carries ~22 significant bits of q against the exact fp16 KV;
 //   C  online softmax in the exp2 domain, P stored as fp16;
 //   D  O += P V on tensor cores, O held in registers (fp32).
+// This mma.sync kernel is the alternative path (CSA_ATTN_MMA_SYNC=1); by
+// default every head count runs the tcgen05 kernel of attn_tc.cu.
 #include <cstdlib>
 
 #include "common.cuh"
@@ -489,7 +491,7 @@ static AttnPlan plan_attn(const csa_attn_args* a, int share) {
   // at least two tiles per split on the mma.sync kernel (each split reloads q
   // and writes a partial O); the tcgen05 kernel takes single tiles, its
   // per-split cost is small next to a tile's latency
-  const int by_tiles = (a->H == 64 && use_tc_attention()) ? n_tiles : (n_tiles + 1) / 2;
+  const int by_tiles = use_tc_attention() ? n_tiles : (n_tiles + 1) / 2;
   if (want > by_tiles) want = by_tiles;
   if (want < 1) want = 1;
   if (want > n_tiles) want = n_tiles > 0 ? n_tiles : 1;
@@ -525,7 +527,7 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-// CSA_ATTN_MMA_SYNC=1 selects the mma.sync kernel for 64 heads too (both
+// CSA_ATTN_MMA_SYNC=1 selects the mma.sync kernel for every head count (both
 // kernels are kept: the tcgen05 one is the default).
 static bool use_tc_attention() {
   static int v = -1;
@@ -537,11 +539,12 @@ static bool use_tc_attention() {
 }
 
 
-// 64 heads run on the tcgen05 kernel; other head counts on the mma.sync kernel.
-static cudaError_t launch_attn_64_tc(AttnParams& p, const void* q2, cudaStream_t stream) {
+// Every head count runs on the tcgen05 kernel (the mma.sync kernel stays as
+// the CSA_ATTN_MMA_SYNC=1 alternative).
+static cudaError_t launch_attn_tc_any(AttnParams& p, const void* q2, cudaStream_t stream) {
   AttnTcParams t;
   t.q2 = static_cast<const uint8_t*>(q2);
-  t.B = p.B; t.n_q = p.n_q; t.q = p.q; t.kv = p.kv; t.kv_row_stride = p.kv_row_stride;
+  t.B = p.B; t.n_q = p.n_q; t.H = p.H; t.q = p.q; t.kv = p.kv; t.kv_row_stride = p.kv_row_stride;
   t.kv_batch_stride = p.kv_batch_stride; t.idx = p.idx; t.K = p.K; t.win = p.win;
   t.win_row_stride = p.win_row_stride; t.win_batch_stride = p.win_batch_stride; t.n_win = p.n_win;
   t.scale_log2 = p.scale_log2; t.sink = p.sink; t.out = p.out; t.lse = p.lse; t.n_entries = p.n_entries;
@@ -554,14 +557,14 @@ static cudaError_t launch_attn_64_tc(AttnParams& p, const void* q2, cudaStream_t
   if (e != cudaSuccess) return e;
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, 64), dim3(kCombThreads), 0, stream, p);
+    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, p.H), dim3(kCombThreads), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();
 }
 
-// True when these arguments run on the tcgen05 kernel (which can take q
-// already staged by a layer stack's prologue).
+// True when these arguments can take q already staged by a layer stack's
+// prologue (64 heads on the tcgen05 kernel).
 bool attn_tc_path(const csa_attn_args* a) { return a->H == 64 && use_tc_attention(); }
 
 cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t stream, const void* q2, int share) {
@@ -585,11 +588,12 @@ cudaError_t run_sparse_attn(const csa_attn_args* a, void* ws, cudaStream_t strea
     p.part_o = static_cast<float*>(ws);
     p.part_ml = p.part_o + tok * pl.n_splits * a->H * kD;
   }
+  if (a->H != 16 && a->H != 32 && a->H != 64) return cudaErrorInvalidValue;
+  if (use_tc_attention()) return launch_attn_tc_any(p, q2, stream);
   switch (a->H) {
     case 16: return launch_attn_h<16>(p, stream);
     case 32: return launch_attn_h<32>(p, stream);
-    case 64: return use_tc_attention() ? launch_attn_64_tc(p, q2, stream) : launch_attn_h<64>(p, stream);
-    default: return cudaErrorInvalidValue;
+    default: return launch_attn_h<64>(p, stream);
   }
 }
 

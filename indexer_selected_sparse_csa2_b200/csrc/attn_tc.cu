@@ -1,5 +1,7 @@
-// Sparse MLA attention on the 5th-generation tensor cores (tcgen05), for 64
-// query heads (the shape of the step's attention layers).
+// Sparse MLA attention on the 5th-generation tensor cores (tcgen05), built
+// for 64 query heads (the shape of the step's attention layers); 16 or 32
+// heads run the same kernel with the query rows of heads >= H left zero and
+// only heads < H written.
 //
 // Same function as sparse_attn_mma_kernel (MLA over the Top-K selected FP4
 // entries plus the FP8 window, K = V = the 512-wide latent; Model techniques
@@ -236,7 +238,8 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   // r = 2h + part holds the pair of channels (8g + (j & 3), 8g + (j & 3) + 4),
   // g = j / 4; lane quarter qq is written by warps qq, qq + 4 and qq + 8, four
   // 16-column stores each.
-  const float* qg = p.q + (int64_t)bt * kAtH * kD;
+  const int H = p.H;                        // 16, 32 or 64 heads; rows of heads >= H stay zero
+  const float* qg = p.q + (int64_t)bt * H * kD;
   if (p.q2) {
     // q staged by the stack prologue: copy rows into TMEM, the rest into shared memory
     // warps 0-3 (one TMEM lane quarter each) move the tensor-memory part
@@ -272,12 +275,12 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     const int qq = warp & 3, wr = warp >> 2;
     const int r = 32 * qq + lane, h = r >> 1;
     const bool lo = r & 1;
-    const float4* qrow = reinterpret_cast<const float4*>(qg + (int64_t)h * kD);
+    const float4* qrow = reinterpret_cast<const float4*>(qg + (int64_t)(h < H ? h : 0) * kD);
 #pragma unroll 1
     for (int u = 4 * wr; u < 4 * wr + 4; ++u) {         // columns 16u .. 16u + 15 = channels 32u .. 32u + 31
       float4 f[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) f[k] = qrow[8 * u + k];
+      for (int k = 0; k < 8; ++k) f[k] = h < H ? qrow[8 * u + k] : make_float4(0.f, 0.f, 0.f, 0.f);
       uint32_t v[16];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
@@ -300,9 +303,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       const int i = tid + t * kAtThreads;
       if (i < 128 * 16) {
         const int r = i >> 4, kb = (i >> 3) & 1, c8 = i & 7;
-        const float4* src = reinterpret_cast<const float4*>(qg + (int64_t)(r >> 1) * kD + 384 + 64 * kb + 8 * c8);
-        f[2 * t] = src[0];
-        f[2 * t + 1] = src[1];
+        const bool live = (r >> 1) < H;
+        const float4* src = reinterpret_cast<const float4*>(qg + (int64_t)(live ? r >> 1 : 0) * kD + 384 + 64 * kb + 8 * c8);
+        f[2 * t] = live ? src[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+        f[2 * t + 1] = live ? src[1] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
       float scl = 1.f;
       if (p.n_splits == 1) {
         float m0 = m_run, l0 = l_run;
-        if (p.sink) {
+        if (p.sink && h < H) {
           const float s0 = p.sink[h] * kAtLog2e;
           const float n0 = fmaxf(m0, s0);
           l0 = (l0 > 0.f ? l0 * exp2f(m0 - n0) : 0.f) + (s0 == -INFINITY ? 0.f : exp2f(s0 - n0));
@@ -612,9 +616,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
         } else {
           scl = l0 > 0.f ? 1.f / l0 : 0.f;
         }
-        if (p.lse) p.lse[(int64_t)bt * kAtH + h] = l0 > 0.f ? (m0 + log2f(l0)) * kAtLn2 : -INFINITY;
-      } else {
-        *reinterpret_cast<float2*>(p.part_ml + (((int64_t)bt * p.n_splits + split) * kAtH + h) * 2) =
+        if (p.lse && h < H) p.lse[(int64_t)bt * H + h] = l0 > 0.f ? (m0 + log2f(l0)) * kAtLn2 : -INFINITY;
+      } else if (h < H) {
+        *reinterpret_cast<float2*>(p.part_ml + (((int64_t)bt * p.n_splits + split) * H + h) * 2) =
             make_float2(m_run, l_run);
       }
       S.scl[h] = scl;
@@ -653,9 +657,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
             o[hd] = __float_as_uint((d & 1) ? v * k.x - pv * k.y : v * k.x + pv * k.y);
           }
         }
-        const int64_t base = (int64_t)bt * kAtH * kD + d;
+        const int64_t base = (int64_t)bt * H * kD + d;
 #pragma unroll
-        for (int hd = 0; hd < kAtH; ++hd) store_out1(p.out, p.out_bf16, base + (int64_t)hd * kD, __uint_as_float(o[hd]));
+        for (int hd = 0; hd < kAtH; ++hd)
+          if (hd < H) store_out1(p.out, p.out_bf16, base + (int64_t)hd * kD, __uint_as_float(o[hd]));
       }
     } else if (!ok || nt == 0) {
       *S.o_bad = 1;
@@ -692,7 +697,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      bulk_store(p.part_o + ((int64_t)bt * p.n_splits + split) * kAtH * kD, S.kv, (uint32_t)(kAtH * kD * 4));
+      bulk_store(p.part_o + ((int64_t)bt * p.n_splits + split) * H * kD, S.kv, (uint32_t)(H * kD * 4));
       bulk_commit();
       bulk_wait_read();                    // the CTA's shared memory must outlive the copy's reads
     }

@@ -8,6 +8,7 @@ namespace csa {
 
 struct AttnTcParams {
   int B, n_q;
+  int H;                      // 16, 32 or 64 query heads (the kernel runs 64, rows past H are zero)
   const float* q;
   const uint8_t* kv;
   int64_t kv_row_stride, kv_batch_stride;
