@@ -9,7 +9,8 @@
 //
 // One warp encodes one 512-channel row; lane l owns channels [16l, 16l+16),
 // i.e. exactly one FP4 scale block, or half of one FP8 scale block.  Rows are
-// read with 128-bit loads and written with 64/128-bit stores.
+// read and written with 128-bit accesses (FP4 codes and scales gathered across
+// lanes by shuffles).
 #include "common.cuh"
 #include "quant.cuh"
 #include "q2.cuh"
@@ -44,7 +45,10 @@ CSA_DEV void load16(const void* row, int lane, float (&x)[16]) {
 }
 
 // Lane `lane` of a warp encodes channels [16 lane, 16 lane + 16) of one FP4
-// entry (one scale block) from values in registers.
+// entry (one scale block) from values in registers.  Called by all 32 lanes
+// of a warp for one entry: the entry is written with 16-byte stores (each
+// even lane stores its codes and its odd neighbour's, lanes 0 and 16 the 32
+// scale bytes).
 CSA_DEV void encode_fp4_vals(const float (&x)[16], int lane, uint8_t* out) {
   float amax = 0.f;
 #pragma unroll
@@ -60,8 +64,19 @@ CSA_DEV void encode_fp4_vals(const float (&x)[16], int lane, uint8_t* out) {
       packed[i >> 2] |= b << (8 * (i & 3));
     }
   }
-  *reinterpret_cast<uint2*>(out + 8 * lane) = make_uint2(packed[0], packed[1]);
-  out[256 + lane] = (uint8_t)s_code;
+  const uint32_t n0 = __shfl_xor_sync(0xffffffffu, packed[0], 1);
+  const uint32_t n1 = __shfl_xor_sync(0xffffffffu, packed[1], 1);
+  if ((lane & 1) == 0) *reinterpret_cast<uint4*>(out + 8 * lane) = make_uint4(packed[0], packed[1], n0, n1);
+  // scale bytes: lane 4w gathers the word of lanes 4w .. 4w + 3, then lanes
+  // 0 and 16 gather four words each
+  uint32_t word = s_code;
+  word |= __shfl_down_sync(0xffffffffu, s_code, 1) << 8;
+  word |= __shfl_down_sync(0xffffffffu, s_code, 2) << 16;
+  word |= __shfl_down_sync(0xffffffffu, s_code, 3) << 24;
+  uint32_t w4[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) w4[k] = __shfl_sync(0xffffffffu, word, (lane & 16) + 4 * k);
+  if ((lane & 15) == 0) *reinterpret_cast<uint4*>(out + 256 + lane) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
 }
 
 // One warp encodes row `row` of the source into one FP4 entry.
