@@ -413,7 +413,12 @@ size_t csa_layer_workspace_size(const csa_layer_desc* layers, int32_t n_layers) 
 // Host-side streams and events the stack uses to run independent layers
 // concurrently (created once per device; no device memory).  Under stream
 // capture the fork / join below becomes graph edges.
-constexpr int kAuxStreams = 8;
+// Auxiliary streams per device: the last stages the decode queries, the
+// others carry layers 1, 2, ... in turn.  Enough that the independent chains
+// of a deep stack (a 40-layer stack has 4 Full layers and their Reuse layers)
+// rarely queue behind one another on a shared stream.
+constexpr int kAuxStreams = 32;
+constexpr int kLayerStreams = kAuxStreams - 1;
 constexpr int kMaxStackLayers = 64;
 static_assert(sizeof(csa_step_sync::layer_done) / sizeof(void*) == kMaxStackLayers, "csa_step_sync layout");
 struct StackStreams {
@@ -562,8 +567,8 @@ csa_status csa_layer_step_sync(const csa_layer_desc* layers, int32_t n_layers, v
       csa_attn_args at{};
       resolve_layer(layers, i, &ix, &at);
       const csa_layer_desc& L = layers[i];
-      if (i > 0) used[(i - 1) % kAuxStreams] = true;
-      cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kAuxStreams];
+      if (i > 0) used[(i - 1) % kLayerStreams] = true;
+      cudaStream_t ls = i == 0 ? st : SS->aux[(i - 1) % kLayerStreams];
       if (i > 0 && cudaStreamWaitEvent(ls, SS->pro, 0) != cudaSuccess) return CSA_ERR_CUDA;
       uint8_t* region = base + reg_off;
       const int share = attn_share(layers, n_layers, i);
