@@ -5,7 +5,7 @@
 
 namespace csa {
 
-constexpr int kMaxBatchJobs = 48;   // 48 x 72-byte jobs: the launch's parameters stay under 4 KB
+constexpr int kMaxBatchJobs = 24;
 // Batch job format (besides the csa_kv_format values): stage a token's 64-head
 // attention query for the tcgen05 attention kernel (q2.cuh); n_rows = tokens
 // x 64 heads, src = fp32 queries [tokens][64][512], dst = [tokens][128 KB].
@@ -31,8 +31,6 @@ struct QuantBatch {
   uint4* zero_ptr;         // optional range cleared by the same launch
   int64_t zero_n16;        // its size in 16-byte words
 };
-
-static_assert(sizeof(QuantBatch) <= 4000, "quant_batch_kernel parameters must fit 4 KB");
 
 // Warp units a job of this format and shape takes.
 int64_t quant_batch_units(int fmt, int64_t n_rows, int dim);
