@@ -175,7 +175,9 @@ CSA_DEV void mma_e4m3_16832_cs(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t
 template <int MODE, int CL>
 __global__ void __launch_bounds__(kCsThreads, 1) cluster_select_kernel(CsJobs jobs, CsPool pp) {
   constexpr bool POOL = MODE != kCsRows;
-  pdl_enter();
+  // shared-memory setup and the cluster's first arrival overlap the previous
+  // kernel; every global read comes after the wait below
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t cs_raw[];
   CsSmem& S = *reinterpret_cast<CsSmem*>(cs_raw);
   const CsRow& J = jobs.j[blockIdx.z];
@@ -195,6 +197,7 @@ __global__ void __launch_bounds__(kCsThreads, 1) cluster_select_kernel(CsJobs jo
   __syncthreads();
   // peers write into this CTA's shared memory only after the matching wait
   cluster_arrive();
+  pdl_wait();
 
   const int64_t nrow = POOL ? min((int64_t)pp.pool_len[b], J.n) : (J.n_row ? min((int64_t)J.n_row[b], J.n) : J.n);
   const int64_t run = J.run;
