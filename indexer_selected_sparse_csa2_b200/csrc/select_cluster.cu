@@ -8,7 +8,7 @@
 // ("2048-block x 8-position candidate pool") is the same selection over block
 // maxima, expanded to the blocks' positions.
 //
-// One cluster of 8 CTAs (16 for rows over 2^18 slots) per (row, job).  Warp w
+// One cluster of 8 CTAs (16 for rows over 2^16 slots) per (row, job).  Warp w
 // of CTA c scans the run [(32c + w) * run, +run) of the row, 4 slots per lane
 // per 128-slot step.
 //   1. the first-level bin beta holding the K-th largest order key, and r,
@@ -54,7 +54,7 @@ constexpr int kCsGatherCap = 8192;     // keys of bin beta gathered in CTA 0 (fa
 constexpr int kCsWarpCap = 192;        // slots of bin >= beta listed per warp
 constexpr int kCsBatch = 4;            // 128-slot steps whose loads are in flight together
 constexpr int kCsSliceCap = 8192;      // pool variants: values per CTA in shared memory
-constexpr int kCsLongRow = 1 << 18;    // rows above this use clusters of 16 CTAs, else 8
+constexpr int kCsLongRow = 1 << 16;    // rows above this use clusters of 16 CTAs, else 8
 constexpr int kCsMaxCluster = 16;
 
 enum CsMode : int { kCsRows = 0, kCsPoolScore = 1, kCsPoolGather = 2 };
