@@ -411,15 +411,29 @@ __global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p
   }
   const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
   if (threadIdx.x < 32) {
-    float M = sk;
-    for (int s = threadIdx.x; s < S; s += 32) M = fmaxf(M, p.part_ml[(((int64_t)bt * S + s) * H + h) * 2]);
+    // (m, l) of splits lane and lane + 32 read once into registers (splits
+    // past 64 are read again below)
+    float2 ml2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = threadIdx.x + 32 * k;
+      ml2[k] = s < S ? *reinterpret_cast<const float2*>(p.part_ml + (((int64_t)bt * S + s) * H + h) * 2)
+                     : make_float2(-INFINITY, 0.f);
+    }
+    float M = fmaxf(sk, fmaxf(ml2[0].x, ml2[1].x));
+    for (int s = threadIdx.x + 64; s < S; s += 32) M = fmaxf(M, p.part_ml[(((int64_t)bt * S + s) * H + h) * 2]);
     M = warp_max(M);
     float L = 0.f;
-    for (int s = threadIdx.x; s < S; s += 32) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = threadIdx.x + 32 * k;
+      const float w = (ml2[k].x == -INFINITY) ? 0.f : exp2f(ml2[k].x - M);
+      L += ml2[k].y * w;
+      if (s < S) wgt_s[s] = w;
+    }
+    for (int s = threadIdx.x + 64; s < S; s += 32) {
       const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (((int64_t)bt * S + s) * H + h) * 2);
-      const float w = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-      L += ml.y * w;
-      if (s < 64) wgt_s[s] = w;
+      L += ml.y * ((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M));
     }
     L = warp_sum(L);
     if (threadIdx.x == 0) {

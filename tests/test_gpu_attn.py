@@ -77,6 +77,7 @@ def _oracle(kv, win, q, idx, n_win, scale, sk=None):
     (1, 1, 16, 300, 1, 0, None),           # a single selected entry, no window
     (1, 40, 64, 20000, 2048, 128, None),   # prefill-like: 40 tokens, 68 tiles each
     (1, 2, 64, 3000, 1000, 100, None),     # K and window not multiples of a tile
+    (1, 1, 64, 20000, 8192, 128, None),    # 130 tiles, more than 64 splits to merge
 ])
 def test_sparse_attention(csa, B, n_q, H, T, K, n_win, valid):
     scale = float(np.float32(1 / np.sqrt(512)))
