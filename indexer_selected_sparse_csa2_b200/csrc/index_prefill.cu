@@ -128,6 +128,15 @@ CSA_DEV int64_t pf_tile(const PfParams& p, const PfItem& x, int64_t i) {
   return first + i * kSampleStride;
 }
 
+// Twice the ReLU of two head dots, x + |x| (exact: 2x for x > 0, +0
+// otherwise), as one packed fp32x2 add on the FMA pipe; the head weights are
+// halved to match, so w * relu(x) = (w / 2) * (x + |x|) is the same product
+// and every fused multiply-add rounds as with max(x, 0).
+CSA_DEV float2 relu2(uint32_t a, uint32_t b) {
+  const float2 x = make_float2(__uint_as_float(a), __uint_as_float(b));
+  return __fadd2_rn(x, make_float2(fabsf(x.x), fabsf(x.y)));
+}
+
 template <int MODE>   // 0 = sample pass, 1 = main pass (p.mode must match)
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
@@ -219,10 +228,14 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
       float tau[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) tau[k] = (MODE == 1 && k < nlive) ? p.tau[row0 + k] : INFINITY;
-      // the group's 8 x 8 head weights stay in registers for the whole item
+      // the group's 8 x 8 head weights stay in registers for the whole item,
+      // halved: w * relu(x) is computed as (w / 2) * (x + |x|) (see relu2)
       float2 wr[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) wr[k] = *reinterpret_cast<const float2*>(S.wts + qg * 64 + 2 * k);
+      for (int k = 0; k < 32; ++k) {
+        const float2 v = *reinterpret_cast<const float2*>(S.wts + qg * 64 + 2 * k);
+        wr[k] = make_float2(0.5f * v.x, 0.5f * v.y);
+      }
       const int kc = (int)(x.kt0 / kPfChunkTiles);
       uint2* cand_base = p.cand + (row0 * p.kchunks + kc) * (int64_t)p.chunk_cap;
       const int nt = (int)n_t;
@@ -249,14 +262,10 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
           for (int kk = 0; kk < 4; ++kk) {
             const int k = 4 * hf + kk;
             const uint32_t* rr = r32 + 8 * kk;
-            float2 acc = __fmul2_rn(wr[4 * k], make_float2(fmaxf(__uint_as_float(rr[0]), 0.f),
-                                                           fmaxf(__uint_as_float(rr[1]), 0.f)));
-            acc = __ffma2_rn(wr[4 * k + 1],
-                             make_float2(fmaxf(__uint_as_float(rr[2]), 0.f), fmaxf(__uint_as_float(rr[3]), 0.f)), acc);
-            acc = __ffma2_rn(wr[4 * k + 2],
-                             make_float2(fmaxf(__uint_as_float(rr[4]), 0.f), fmaxf(__uint_as_float(rr[5]), 0.f)), acc);
-            acc = __ffma2_rn(wr[4 * k + 3],
-                             make_float2(fmaxf(__uint_as_float(rr[6]), 0.f), fmaxf(__uint_as_float(rr[7]), 0.f)), acc);
+            float2 acc = __fmul2_rn(wr[4 * k], relu2(rr[0], rr[1]));
+            acc = __ffma2_rn(wr[4 * k + 1], relu2(rr[2], rr[3]), acc);
+            acc = __ffma2_rn(wr[4 * k + 2], relu2(rr[4], rr[5]), acc);
+            acc = __ffma2_rn(wr[4 * k + 3], relu2(rr[6], rr[7]), acc);
             sc[k] = acc.x + acc.y;
           }
         }
