@@ -165,13 +165,6 @@ CSA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-CSA_DEV void tmem_ld16f(uint32_t taddr, float* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
-        "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15])
-      : "r"(taddr));
-}
 CSA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // 32 consecutive columns of this warp's 32 lanes in one instruction.
 CSA_DEV void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
@@ -239,18 +232,6 @@ CSA_DEV uint32_t dsmem_ld(uint32_t addr) {
   return v;
 }
 
-CSA_DEV void dsmem_st_v2f(uint32_t addr, float2 v) {
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
-}
-// No memory clobber: a caller that issues several of these back to back keeps
-// them all in flight (ordering against peers' writes comes from the cluster
-// barrier, itself a compiler memory barrier).
-CSA_DEV float4 dsmem_ld_v4f(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
 
 // ------------------------------------------------------------- descriptors --
 // Shared-memory matrix descriptor, K-major, 64-byte swizzle: rows of 64 bytes,
