@@ -42,10 +42,9 @@
 // probabilities by 2^7 in P, which leaves S and O unchanged.  Window entries
 // are staged unscaled.
 //
-// With several splits per token the partial O^T (unnormalised) is copied from
-// TMEM into the freed entry-tile buffers as [head][channel] fp32 rows and
-// written to global memory by one 128 KB bulk copy; attn_combine merges the
-// splits.  The kernel triggers its dependents at once and does its prologue
+// With several splits per token the partial O^T (unnormalised) is written
+// from TMEM to global memory as [head][channel] fp32 rows (coalesced per
+// head); attn_combine merges the splits.  The kernel triggers its dependents at once and does its prologue
 // (barrier setup, TMEM allocation, the query staging from caller memory or
 // from the stack's staging buffer, which a full event dependency orders)
 // before it waits for the previous kernel on its stream, so the prologue
@@ -669,13 +668,15 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
   if (p.n_splits > 1) {
     // ------------------------------------------------------ partial O^T
     // the softmax warps have seen the last PV retire; warps w and w + 4 share
-    // TMEM lane quarter w & 3 and copy chunks {0, 1} and {2, 3} into the freed
-    // entry buffers as [head][channel] rows, then one bulk copy writes them
+    // TMEM lane quarter w & 3 and write chunks {0, 1} and {2, 3} as
+    // [head][channel] rows straight from their TMEM rows: per head a warp
+    // stores 32 neighbouring channels (128 contiguous bytes).  Staging the
+    // rows in shared memory for one bulk copy was slower: the copy moved the
+    // 128 KB no faster than these stores, after the staging.
     __syncthreads();
     if (warp < 8) {
       const int qq = warp & 3, cb = 2 * (warp >> 2);
       const bool valid = *S.o_bad == 0;
-      float* stage = reinterpret_cast<float*>(S.kv);
       tc_fence_after();
 #pragma unroll 1
       for (int cc = 0; cc < 2; ++cc) {
@@ -690,16 +691,11 @@ __global__ void __launch_bounds__(kAtThreads, 1) sparse_attn_tc_kernel(AttnTcPar
 #pragma unroll
           for (int k = 0; k < 64; ++k) o[k] = 0u;
         }
+        float* po = p.part_o + ((int64_t)bt * p.n_splits + split) * H * kD + d;
 #pragma unroll
-        for (int hd = 0; hd < kAtH; ++hd) stage[hd * kD + d] = __uint_as_float(o[hd]);
+        for (int hd = 0; hd < kAtH; ++hd)
+          if (hd < H) po[(int64_t)hd * kD] = __uint_as_float(o[hd]);
       }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      bulk_store(p.part_o + ((int64_t)bt * p.n_splits + split) * H * kD, S.kv, (uint32_t)(H * kD * 4));
-      bulk_commit();
-      bulk_wait_read();                    // the CTA's shared memory must outlive the copy's reads
     }
   }
 #undef CSA_AT_FETCH

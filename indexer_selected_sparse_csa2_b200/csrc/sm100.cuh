@@ -89,17 +89,6 @@ CSA_DEV void cp_async16(uint32_t dst_smem, const void* src) {
 }
 CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-// Untiled bulk copy this CTA's shared memory -> global (same alignment rules),
-// tracked as a bulk async-group of the issuing thread.
-CSA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-               ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
-}
-CSA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until every bulk async-group of this thread has read its source (the
-// shared memory may then be reused or released); the writes themselves are
-// visible to work ordered after the kernel, as any store of the kernel is.
-CSA_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Untiled bulk copy global -> this CTA's shared memory (no multicast):
 // addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
 CSA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
