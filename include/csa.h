@@ -156,7 +156,8 @@ typedef struct {
    * (architecture database, indexer K: E2M1 with one E8M0 scale per 32
    * channels; techniques map: 32 heads x 128): d_I = 128, H_I = 32, decode
    * scans only (no pool search); `keys` holds the E2M1 codes (64 bytes per
-   * key, even channel in the low nibble) and `key_scales` the 4 exponent
+   * key, even channel in the low nibble; `keys` 32-byte aligned and both key
+   * strides multiples of 32, else CSA_ERR_ALIGNMENT) and `key_scales` the 4 exponent
    * bytes (e + 127, block order) of key s at key_scales +
    * b*key_scale_batch_stride + s*key_scale_row_stride (strides multiples of
    * 4).  Block b of the key contributes 2^e_b * <q block b, E2M1 codes>. */

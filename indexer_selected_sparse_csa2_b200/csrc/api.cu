@@ -76,6 +76,8 @@ static csa_status check_index(const csa_index_args* a) {
     if (a->key_scale_row_stride < 4 || ((uintptr_t)a->key_scales & 3) || (a->key_scale_row_stride & 3) ||
         (a->key_scale_batch_stride & 3))
       return CSA_ERR_ALIGNMENT;
+    // the packed 4-bit copy into the tensor cores' operand layout
+    if (((uintptr_t)a->keys & 31) || (a->key_row_stride & 31) || (a->key_batch_stride & 31)) return CSA_ERR_ALIGNMENT;
   } else if (a->key_format != CSA_KEY_E4M3) {
     return CSA_ERR_INVALID_ARG;
   } else if (a->H_I < 1 || a->H_I > 8 || a->d_I != kDI) {
@@ -336,15 +338,17 @@ static size_t layer_region_bytes(const csa_layer_desc& L, const csa_index_args& 
 // The first key row of `ix` that the stack's prologue (every layer's append
 // jobs) writes, for the full scan that overlaps the prologue: rows below it may
 // be read before the prologue ends.  -1 (wait first) when a job writes the
-// query or the head weights, or when the keys are not a plain E4M3 row cache.
+// query or the head weights.  MXFP4 keys are read only after the wait (0: no
+// row early, the query and weights may be).
 static int64_t prologue_safe_rows(const csa_layer_desc* layers, int32_t n_layers, const csa_index_args& ix) {
-  if (ix.key_format != CSA_KEY_E4M3 || ix.pool || ix.n_q != 1 || ix.T <= 0) return -1;
+  const bool mx = ix.key_format == CSA_KEY_MXFP4;
+  if ((ix.key_format != CSA_KEY_E4M3 && !mx) || ix.pool || ix.n_q != 1 || ix.T <= 0) return -1;
   const int64_t bs = ix.key_batch_stride ? ix.key_batch_stride : ix.key_row_stride * ix.T;
   const uintptr_t k0 = reinterpret_cast<uintptr_t>(ix.keys);
   const uintptr_t k1 = k0 + (uintptr_t)((ix.B - 1) * bs + ix.T * ix.key_row_stride);
-  const uintptr_t q0 = reinterpret_cast<uintptr_t>(ix.q), q1 = q0 + (uintptr_t)ix.B * ix.H_I * kDI;
+  const uintptr_t q0 = reinterpret_cast<uintptr_t>(ix.q), q1 = q0 + (uintptr_t)ix.B * ix.H_I * ix.d_I;
   const uintptr_t w0 = reinterpret_cast<uintptr_t>(ix.w), w1 = w0 + (uintptr_t)ix.B * ix.H_I * 4;
-  int64_t safe = ix.T;
+  int64_t safe = mx ? 0 : ix.T;
   for (int32_t i = 0; i < n_layers; ++i) {
     for (int k = 0; k < 3; ++k) {
       const csa_quant_job& q = layers[i].append[k];
@@ -356,7 +360,7 @@ static int64_t prologue_safe_rows(const csa_layer_desc* layers, int32_t n_layers
         const uintptr_t a1 = a0 + (uintptr_t)rb;
         if (a0 < q1 && a1 > q0) return -1;
         if (a0 < w1 && a1 > w0) return -1;
-        if (a0 >= k1 || a1 <= k0) continue;
+        if (mx || a0 >= k1 || a1 <= k0) continue;
         // the rows this write touches (from its first and last byte)
         for (uintptr_t a : {a0 < k0 ? k0 : a0, (a1 > k1 ? k1 : a1) - 1}) {
           const int64_t off = (int64_t)(a - k0);

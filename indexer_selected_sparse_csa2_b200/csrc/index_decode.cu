@@ -208,7 +208,7 @@ static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
                             int64_t nb, int64_t safe_rows, cudaStream_t stream);
 cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
-                            int64_t nb, cudaStream_t stream);
+                            int64_t nb, bool q_early, cudaStream_t stream);
 
 // Pool searches whose slots fit the fused cluster kernel score and select in
 // one launch and need no workspace.
@@ -323,7 +323,7 @@ cudaError_t run_index_decode(const csa_index_args* a, void* ws, cudaStream_t str
     p.hist = w.hist;
     e = launch_score_decode(p, B, stream);
   } else if (a->key_format == CSA_KEY_MXFP4) {
-    e = launch_score_mx(a, scores, pos_hist, w.bmax, w.bhist, nb, stream);
+    e = launch_score_mx(a, scores, pos_hist, w.bmax, w.bhist, nb, hists && safe_rows >= 0, stream);
   } else {
     e = launch_score_tc(a, scores, pos_hist, w.bmax, w.bhist, nb, hists ? safe_rows : -1, stream);
   }

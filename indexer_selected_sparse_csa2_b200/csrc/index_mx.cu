@@ -7,18 +7,23 @@
 //   S[s] = sum_j w[j] * relu( sum_b 2^(e[s,b]) * <q[j, block b], k[s, block b]> )
 // where k is the key's E2M1 codes and e its block exponents.
 // Keys sit in two planes: codes [B][T][64 B] and exponent bytes [B][T][4].
-//   warp 0     TMA producer: 128-key x 64-byte code tiles (64-byte swizzle)
-//              into a 12-stage ring (96 KB in flight: one CTA per SM);
+//   warp 0     TMA producer: 128-key tiles of the code plane, copied with the
+//              packed 4-bit tensor-map type that gives every 16 codes (8
+//              bytes) a 16-byte slot in shared memory: the layout in which
+//              tcgen05.mma kind::f8f6f4 reads E2M1 operands (one byte of
+//              address space per element), 128-byte swizzled; 4 stages;
 //   warp 1     MMA issuer: per tile, one tcgen05.mma kind::f8f6f4 per 32-channel
-//              block (M = 128 keys, N = 32 heads, K = 32) into its own TMEM
-//              accumulator (4 x 32 columns per tile, four tiles in flight);
-//   warps 2-9  decode: two threads per key (64 channels each), E2M1 codes ->
-//              E4M3 bytes (every E2M1 value is an E4M3 value) into a
-//              128-byte-swizzled K-major tile, four tiles in flight;
-//   warps 10-13 epilogue: one key per thread, the 4 x 32 block dots from TMEM,
-//              times 2^e per block, ReLU, head weights, the fp32 score, the
-//              first-level Top-K histogram and, when building the pool, the
-//              block maxima.
+//              block (A = E2M1 keys, M = 128; B = E4M3 queries, N = 32 heads;
+//              K = 32) into its own TMEM accumulator (4 x 32 columns per
+//              tile, two tiles in flight);
+//   warps 2-5  epilogue: one key per thread, the 4 x 32 block dots from
+//              TMEM, times 2^e per block, ReLU, head weights, the fp32 score,
+//              the first-level Top-K histogram and, when building the pool,
+//              the block maxima.
+// No thread converts a code: the copy engine spreads them and the tensor
+// cores read E2M1 as it is stored.  Two CTAs share each SM (about 100 KB of
+// shared memory and 256 TMEM columns each): one CTA's copies land one tile
+// per ~0.43 us, so a second CTA doubles the loads in flight per SM.
 // All waits are bounded (sm100.cuh).
 #include "sm100.cuh"
 #include "select.cuh"
@@ -27,18 +32,17 @@ namespace csa {
 
 constexpr int kMxRows = 128;                    // keys per tile
 constexpr int kMxHeads = 32;
-constexpr int kMxStages = 12;                 // 96 KB of key tiles in flight per SM
-constexpr int kMxStageBytes = kMxRows * 64;     // packed codes, 8 KB
-constexpr int kMxDec = 4;                       // decoded tiles in flight
-constexpr int kMxDecWarps = 8;
-constexpr int kMxDecBytes = kMxRows * 128;      // 16 KB
+constexpr int kMxStages = 4;
+constexpr int kMxStageBytes = kMxRows * 128;    // 16 KB of shared memory per tile (16-byte slot per 16 codes)
+constexpr uint32_t kMxStageTx = kMxRows * 64;   // bytes the copy counts: the packed codes
 constexpr int kMxEpiGroups = 1;
-constexpr int kMxAcc = 4;
+constexpr int kMxAcc = 2;
 constexpr uint32_t kMxTmemCols = 128 * kMxAcc;  // kMxAcc x 4 blocks x 32 heads
-constexpr int kMxEpiWarp0 = 2 + kMxDecWarps;
+constexpr int kMxEpiWarp0 = 2;
 constexpr int kMxThreads = 32 * kMxEpiWarp0 + 128 * kMxEpiGroups;
-constexpr size_t kMxSmemBytes = 1024 + (size_t)kMxStages * kMxStageBytes + (size_t)kMxDec * kMxDecBytes +
-                                kMxHeads * 128 + 2 * kHistBins * 4 + 2 * (kMxStages + kMxDec + kMxAcc) * 8 + 16;
+constexpr size_t kMxSmemBytes = 1024 + (size_t)kMxStages * kMxStageBytes + kMxHeads * 128 + 2 * kHistBins * 4 +
+                                2 * (kMxStages + kMxAcc) * 8 + 16;
+static_assert(2 * (kMxSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
 
 static __device__ int g_mx_error;
 
@@ -55,34 +59,25 @@ struct MxScoreParams {
   uint32_t* bhist;
   int64_t nb;
   int block_len;
+  int q_early;              // q and w may be read before the wait on the previous kernel
 };
 
-// E2M1 magnitude code -> E4M3 byte of the same value: 0, 0.5, 1, 1.5, 2, 3, 4, 6
-constexpr uint32_t kE2M1toE4M3Lo = 0x3C383000u;
-constexpr uint32_t kE2M1toE4M3Hi = 0x4C484440u;
-// Four E2M1 codes (nibbles 0-3 of w) as four E4M3 bytes.
-CSA_DEV uint32_t e2m1x4_to_e4m3(uint32_t w) {
-  const uint32_t mag = __byte_perm(kE2M1toE4M3Lo, kE2M1toE4M3Hi, w & 0x7777u);
-  const uint32_t sgn = ((w & 0x8u) << 4) | ((w & 0x80u) << 8) | ((w & 0x800u) << 12) | ((w & 0x8000u) << 16);
-  return mag | sgn;
-}
-
-__global__ void __launch_bounds__(kMxThreads, 1)
+__global__ void __launch_bounds__(kMxThreads, 2)
 index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p) {
-  pdl_enter();
+  // the set-up (barriers, histogram clearing, TMEM, and the queries when no
+  // appended row of the step writes them) overlaps the previous kernel; keys,
+  // exponents and the global histograms are touched only after the wait
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* stage = base;
-  uint8_t* dec = stage + (size_t)kMxStages * kMxStageBytes;
-  uint8_t* qb = dec + (size_t)kMxDec * kMxDecBytes;
+  uint8_t* qb = stage + (size_t)kMxStages * kMxStageBytes;
   uint32_t* h = reinterpret_cast<uint32_t*>(qb + kMxHeads * 128);
   uint32_t* hb = h + kHistBins;
   uint64_t* bars = reinterpret_cast<uint64_t*>(hb + kHistBins);
-  uint64_t* full = bars;                       // [kMxStages] TMA -> decode
-  uint64_t* empty = full + kMxStages;          // [kMxStages] decode -> TMA (4 warps)
-  uint64_t* dfull = empty + kMxStages;         // [kMxDec] decode -> MMA (4 warps)
-  uint64_t* dempty = dfull + kMxDec;           // [kMxDec] MMA -> decode
-  uint64_t* accf = dempty + kMxDec;            // [kMxAcc] MMA -> epilogue
+  uint64_t* full = bars;                       // [kMxStages] TMA -> MMA
+  uint64_t* empty = full + kMxStages;          // [kMxStages] MMA -> TMA
+  uint64_t* accf = empty + kMxStages;          // [kMxAcc] MMA -> epilogue
   uint64_t* acce = accf + kMxAcc;              // [kMxAcc] epilogue -> MMA (4 warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + kMxAcc);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -94,24 +89,31 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
   const bool build = p.bmax != nullptr;
 
   if (tid == 0) {
-    for (int i = 0; i < kMxStages; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, kMxDecWarps); }
-    for (int i = 0; i < kMxDec; ++i) { mbar_init(dfull + i, kMxDecWarps); mbar_init(dempty + i, 1); }
+    for (int i = 0; i < kMxStages; ++i) { mbar_init(full + i, 1); mbar_init(empty + i, 1); }
     for (int i = 0; i < kMxAcc; ++i) { mbar_init(accf + i, 1); mbar_init(acce + i, 4); }
     fence_mbar_init();
     prefetch_tmap(&tmap);
   }
   for (int i = tid; i < kHistBins; i += kMxThreads) { h[i] = 0; hb[i] = 0; }
   // queries: the B operand, 32 rows of 128 bytes, 128-byte swizzle
-  for (int i = tid; i < kMxHeads * 8; i += kMxThreads) {
-    const int r = i >> 3, c = i & 7;
-    const uint4 v = ld_v4(p.q + ((int64_t)b * kMxHeads + r) * 128 + 16 * c);
-    *reinterpret_cast<uint4*>(qb + r * 128 + ((c ^ (r & 7)) << 4)) = v;
-  }
-  fence_proxy_async_smem();
+  auto stage_q = [&]() {
+    for (int i = tid; i < kMxHeads * 8; i += kMxThreads) {
+      const int r = i >> 3, c = i & 7;
+      const uint4 v = ld_v4(p.q + ((int64_t)b * kMxHeads + r) * 128 + 16 * c);
+      *reinterpret_cast<uint4*>(qb + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+  };
+  if (p.q_early) stage_q();
   if (warp == 1) tmem_alloc(tmem_slot, kMxTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
+  if (!p.q_early) {
+    stage_q();
+    __syncthreads();
+  }
   const uint32_t tbase = *tmem_slot;
 
   if (warp == 0) {
@@ -119,58 +121,27 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
       for (int i = 0; i < n_my; ++i) {
         const int s = i % kMxStages;
         if (!mbar_wait(empty + s, ((uint32_t)(i / kMxStages) & 1u) ^ 1u, &g_mx_error, kErrWaitSmemEmpty)) break;
-        mbar_arrive_expect_tx(full + s, kMxStageBytes);
+        mbar_arrive_expect_tx(full + s, kMxStageTx);
         tma_load_3d(stage + (size_t)s * kMxStageBytes, &tmap, full + s, 0, (int)((tile0 + i) * kMxRows), b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_make(kFmtE4M3, kFmtE4M3, kMxRows, kMxHeads);
+      constexpr uint32_t idesc = idesc_make(kFmtE2M1, kFmtE4M3, kMxRows, kMxHeads);
       const uint32_t qa = smem_u32(qb);
       for (int i = 0; i < n_my; ++i) {
-        const int d = i % kMxDec, a = i % kMxAcc;
-        if (!mbar_wait(dfull + d, (uint32_t)(i / kMxDec) & 1u, &g_mx_error, kErrWaitTmaFull)) break;
+        const int s = i % kMxStages, a = i % kMxAcc;
+        if (!mbar_wait(full + s, (uint32_t)(i / kMxStages) & 1u, &g_mx_error, kErrWaitTmaFull)) break;
         if (!mbar_wait(acce + a, ((uint32_t)(i / kMxAcc) & 1u) ^ 1u, &g_mx_error, kErrWaitAccEmpty)) break;
         tc_fence_after();
-        const uint32_t da = smem_u32(dec + (size_t)d * kMxDecBytes);
+        const uint32_t sa = smem_u32(stage + (size_t)s * kMxStageBytes);
 #pragma unroll
         for (int blk = 0; blk < 4; ++blk)
-          mma_f8f6f4_ss(tbase + (uint32_t)(a * 128 + 32 * blk), desc_k_sw128(da + 32u * blk),
+          mma_f8f6f4_ss(tbase + (uint32_t)(a * 128 + 32 * blk), desc_k_sw128(sa + 32u * blk),
                         desc_k_sw128(qa + 32u * blk), idesc, 0u);
-        mma_commit(dempty + d);
+        mma_commit(empty + s);
         mma_commit(accf + a);
       }
-    }
-  } else if (warp < kMxEpiWarp0) {
-    // ---- decode: threads 2r and 2r + 1 take key row r, packed chunks
-    // {0, 1} and {2, 3} (64 channels each)
-    const int r = (tid - 64) >> 1, hf = (tid - 64) & 1;
-    for (int i = 0; i < n_my; ++i) {
-      const int s = i % kMxStages, d = i % kMxDec;
-      bool ok = __all_sync(0xffffffffu, mbar_wait(full + s, (uint32_t)(i / kMxStages) & 1u, &g_mx_error, kErrWaitTmaFull));
-      if (i >= kMxDec)
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(dempty + d, ((uint32_t)(i / kMxDec) - 1u) & 1u, &g_mx_error,
-                                                     kErrWaitSmemEmpty));
-      if (!ok) break;
-      const uint8_t* src = stage + (size_t)s * kMxStageBytes + r * 64;
-      uint8_t* dst = dec + (size_t)d * kMxDecBytes + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        const int c = 2 * hf + cc;
-        // packed chunk c (channels 32c .. 32c + 31) at its 64-byte-swizzle position
-        const uint4 v = *reinterpret_cast<const uint4*>(src + ((c ^ ((r >> 1) & 3)) << 4));
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {          // 16 channels -> one 16-byte chunk j = 2c + hh
-          const uint32_t w0 = wv[2 * hh], w1 = wv[2 * hh + 1];
-          const int j = 2 * c + hh;
-          *reinterpret_cast<uint4*>(dst + ((j ^ (r & 7)) << 4)) =
-              make_uint4(e2m1x4_to_e4m3(w0), e2m1x4_to_e4m3(w0 >> 16), e2m1x4_to_e4m3(w1), e2m1x4_to_e4m3(w1 >> 16));
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) { mbar_arrive(empty + s); mbar_arrive(dfull + d); }
     }
   } else {
     // ---- epilogue: group g takes tiles g, g + G, ...; warp w reads TMEM
@@ -244,13 +215,14 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
   }
 }
 
-bool make_key_tmap(CUtensorMap* map, const uint8_t* keys, int64_t T, int B, int64_t row_stride,
-                   int64_t batch_stride);
+bool make_key_tmap_e2m1(CUtensorMap* map, const uint8_t* keys, int64_t T, int B, int64_t row_stride,
+                        int64_t batch_stride, int box_rows);
 
 cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
-                            int64_t nb, cudaStream_t stream) {
+                            int64_t nb, bool q_early, cudaStream_t stream) {
   CUtensorMap map;
-  if (!make_key_tmap(&map, a->keys, a->T, a->B, a->key_row_stride, a->key_batch_stride)) return cudaErrorInvalidValue;
+  if (!make_key_tmap_e2m1(&map, a->keys, a->T, a->B, a->key_row_stride, a->key_batch_stride, kMxRows))
+    return cudaErrorInvalidValue;
   MxScoreParams p{};
   p.q = a->q;
   p.w = a->w;
@@ -259,9 +231,9 @@ cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hi
   p.scale_batch_stride = a->key_scale_batch_stride;
   p.T = a->T;
   const int64_t ntiles = (a->T + kMxRows - 1) / kMxRows;
-  // one wave: at most one CTA per SM (rounded down, so that no CTA waits
-  // for a second wave)
-  int64_t ctas_row = kNumSMs / a->B;
+  // one wave of two CTAs per SM (rounded down, so that no CTA waits for a
+  // second wave)
+  int64_t ctas_row = 2 * kNumSMs / a->B;
   if (ctas_row > ntiles) ctas_row = ntiles;
   if (ctas_row < 1) ctas_row = 1;
   p.tiles_per_cta = (int)((ntiles + ctas_row - 1) / ctas_row);
@@ -272,6 +244,7 @@ cudaError_t launch_score_mx(const csa_index_args* a, float* scores, uint32_t* hi
   p.bhist = bhist;
   p.nb = nb;
   p.block_len = a->pool_block_len;
+  p.q_early = q_early ? 1 : 0;
   static SmemAttrOnce attr;
   const cudaError_t ea = attr.set(index_score_mx_kernel, kMxSmemBytes);
   if (ea != cudaSuccess) return ea;

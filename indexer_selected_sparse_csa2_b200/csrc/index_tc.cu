@@ -237,6 +237,24 @@ bool make_key_tmap(CUtensorMap* map, const uint8_t* keys, int64_t T, int B, int6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// E2M1 key codes (64 bytes = 128 codes per key) for kind::f8f6f4 operands:
+// the packed 4-bit type copies every 16 codes into a 16-byte slot (8 bytes of
+// codes, 8 bytes left unwritten), 128-key x 128-code boxes, 128-byte swizzle.
+// The type needs a 32-byte aligned base and 32-byte multiple strides.
+bool make_key_tmap_e2m1(CUtensorMap* map, const uint8_t* keys, int64_t T, int B, int64_t row_stride,
+                        int64_t batch_stride, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  if (batch_stride == 0) batch_stride = row_stride * T;
+  const cuuint64_t dims[3] = {128, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_stride, (cuuint64_t)batch_stride};
+  const cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint8_t*>(keys), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hist, float* bmax, uint32_t* bhist,
                             int64_t nb, int64_t safe_rows, cudaStream_t stream) {
   CUtensorMap map;

@@ -274,6 +274,7 @@ CSA_DEV uint32_t sw128_offset_h(uint32_t r, uint32_t c) {
   return (r >> 3) * 1024u + (r & 7u) * 128u + ((((c >> 3) ^ r) & 7u) << 4) + (c & 7u) * 2u;
 }
 constexpr uint32_t kFmtE4M3 = 0;   // kind::f8f6f4 operand format
+constexpr uint32_t kFmtE2M1 = 5;   // kind::f8f6f4 operand format (4-bit codes in 16-byte slots of 16)
 constexpr uint32_t kFmtF16 = 0;    // kind::f16 operand format
 
 // Byte offset of (row r, byte c) inside 64-byte-swizzled rows.
