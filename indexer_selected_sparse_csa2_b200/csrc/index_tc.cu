@@ -6,7 +6,7 @@
 // DeepSeek-V4.1-Flash, "Indexer-selected sparse attention" row), built the
 // sm_100a way:
 //   warp 0  TMA producer: 128-position x 64-byte key tiles (8 KB, 64-byte
-//           swizzle) into an 8-stage shared-memory ring;
+//           swizzle) into a 5-stage shared-memory ring;
 //   warp 1  MMA issuer: per tile two tcgen05.mma kind::f8f6f4 (M = 128
 //           positions, N = 16 query heads, K = 2 x 32 bytes), fp32
 //           accumulators in TMEM, six accumulator buffers;
@@ -29,7 +29,7 @@ namespace csa {
 
 constexpr int kTcEpiGroups = 3;
 constexpr int kTcThreads = 64 + 128 * kTcEpiGroups;
-constexpr int kTcStages = 8;
+constexpr int kTcStages = 5;
 constexpr int kTcAcc = 2 * kTcEpiGroups;
 constexpr int kTcRows = 128;
 constexpr int kTcN = 16;                              // heads per MMA (8 used, rest zero)
@@ -84,7 +84,7 @@ CSA_DEV TcSmem carve_tc_smem(uint8_t* raw) {
   return s;
 }
 
-__global__ void __launch_bounds__(kTcThreads, 2)
+__global__ void __launch_bounds__(kTcThreads, 3)
 index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p) {
   pdl_trigger();
   const bool pre = p.safe_rows >= 0;
@@ -266,9 +266,11 @@ cudaError_t launch_score_tc(const csa_index_args* a, float* scores, uint32_t* hi
   p.H_I = a->H_I;
   p.T = a->T;
   const int64_t ntiles = (a->T + kTcRows - 1) / kTcRows;
-  // two resident CTAs per SM (about 100 KB of shared memory and 128 TMEM
-  // columns each): twice the loads in flight and epilogue warps per SM
-  int64_t ctas_row = 2 * kNumSMs / a->B;                 // one wave (rounded down)
+  // three resident CTAs per SM (about 75 KB of shared memory, 128 TMEM
+  // columns and 40 registers a thread each): each CTA's copies land at a
+  // bounded rate, so more CTAs per SM keep more of HBM busy (two: 154.5 us
+  // per hier_1m step, three: 153.4 us)
+  int64_t ctas_row = 3 * kNumSMs / a->B;                 // one wave (rounded down)
   if (ctas_row > ntiles) ctas_row = ntiles;
   if (ctas_row < 1) ctas_row = 1;
   p.tiles_per_cta = (int)((ntiles + ctas_row - 1) / ctas_row);
