@@ -380,101 +380,84 @@ __global__ void __launch_bounds__(kAttnThreads, 1) sparse_attn_mma_kernel(AttnPa
   }
 }
 
-// Merge the per-split partial results (log-sum-exp combine): one CTA per
-// (token, head), 128 threads x 4 channels.
-// One CTA per (token, head): 4 groups of 128 threads each take a quarter of
-// the splits for all 512 channels (4 per thread), so a thread keeps all of
-// its partial-O loads in flight at once; the groups' sums meet in shared
-// memory.  Split weights 2^(m_s - M) come from the (max, sum) partials.
-constexpr int kCombThreads = 512;
-constexpr int kCombGroups = kCombThreads / 128;
-__global__ void __launch_bounds__(kCombThreads) attn_combine_kernel(AttnParams p) {
+// Merge the per-split partial results (log-sum-exp combine).  CTA (token,
+// head, c) of 128 threads takes channels [128c, 128c + 128) with no shared
+// memory and at most 64 registers a thread, so that a combine CTA fits on an
+// SM beside one tcgen05 attention CTA (which leaves 8192 registers and no
+// shared memory beyond the per-CTA reservation): one layer's combine runs
+// while later layers' attention CTAs hold the SMs.  Lane group g = lane / 8
+// of each warp takes splits g, g + 4, ... for 8 x 4 channels (its loads in
+// flight together), the four groups' sums meet by shuffles.  Every warp
+// reduces the splits' (max, sum) partials itself (lane s holds splits s and
+// s + 32); split weights 2^(m_s - M) reach the other lanes by shuffles.
+constexpr int kCombThreads = 128;
+constexpr int kCombChunks = kD / 128;          // channel chunks (grid z)
+__global__ void __launch_bounds__(kCombThreads, 8) attn_combine_kernel(AttnParams p) {
   pdl_enter();
   const int bt = blockIdx.x, h = blockIdx.y, H = p.H;
   const int S = p.n_splits;
-  __shared__ float wgt_s[64];
-  __shared__ float inv_s, max_s;
-  __shared__ float4 part[kCombGroups - 1][128];
-  const int grp = threadIdx.x >> 7, t = threadIdx.x & 127;
-  const int d = 4 * t;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, g = lane >> 3;
+  const int d = 128 * blockIdx.z + 4 * (8 * warp + (lane & 7));
   const float* po = p.part_o + ((int64_t)bt * S * H + h) * kD + d;
   const int64_t sstride = (int64_t)H * kD;
-  // this group's splits grp, grp + 4, ...: the first round of partial loads
-  // (up to 10 per thread) goes out before the merge weights are known, so the
-  // two dependent reads overlap
-  constexpr int kR = 10;
+  const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (int64_t)bt * S * H + h;
+  constexpr int kR = 8;
   uint4 v[kR];
 #pragma unroll
   for (int k = 0; k < kR; ++k) {
-    const int s = grp + k * kCombGroups;
+    const int s = g + 4 * k;
     v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
   }
   const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-  if (threadIdx.x < 32) {
-    // (m, l) of splits lane and lane + 32 read once into registers (splits
-    // past 64 are read again below)
-    float2 ml2[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int s = threadIdx.x + 32 * k;
-      ml2[k] = s < S ? *reinterpret_cast<const float2*>(p.part_ml + (((int64_t)bt * S + s) * H + h) * 2)
-                     : make_float2(-INFINITY, 0.f);
-    }
-    float M = fmaxf(sk, fmaxf(ml2[0].x, ml2[1].x));
-    for (int s = threadIdx.x + 64; s < S; s += 32) M = fmaxf(M, p.part_ml[(((int64_t)bt * S + s) * H + h) * 2]);
-    M = warp_max(M);
-    float L = 0.f;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int s = threadIdx.x + 32 * k;
-      const float w = (ml2[k].x == -INFINITY) ? 0.f : exp2f(ml2[k].x - M);
-      L += ml2[k].y * w;
-      if (s < S) wgt_s[s] = w;
-    }
-    for (int s = threadIdx.x + 64; s < S; s += 32) {
-      const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + (((int64_t)bt * S + s) * H + h) * 2);
-      L += ml.y * ((ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M));
-    }
-    L = warp_sum(L);
-    if (threadIdx.x == 0) {
-      if (sk != -INFINITY) L += exp2f(sk - M);
-      inv_s = L > 0.f ? 1.f / L : 0.f;
-      if (p.lse) p.lse[(int64_t)bt * H + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-      max_s = M;
-    }
+  const float2 ml0 = lane < S ? ml[(int64_t)lane * H] : make_float2(-INFINITY, 0.f);
+  const float2 ml1 = lane + 32 < S ? ml[(int64_t)(lane + 32) * H] : make_float2(-INFINITY, 0.f);
+  float M = fmaxf(sk, fmaxf(ml0.x, ml1.x));
+  for (int s = lane + 64; s < S; s += 32) M = fmaxf(M, ml[(int64_t)s * H].x);
+  M = warp_max(M);
+  const float w0 = ml0.x == -INFINITY ? 0.f : exp2f(ml0.x - M);
+  const float w1 = ml1.x == -INFINITY ? 0.f : exp2f(ml1.x - M);
+  float L = ml0.y * w0 + ml1.y * w1;
+  for (int s = lane + 64; s < S; s += 32) {
+    const float2 m2 = ml[(int64_t)s * H];
+    L += m2.y * (m2.x == -INFINITY ? 0.f : exp2f(m2.x - M));
   }
-  __syncthreads();
-  const float M = max_s;
+  L = warp_sum(L);
+  if (sk != -INFINITY) L += exp2f(sk - M);
+  // weight of split s (s differs between lane groups; every lane shuffles)
   auto weight = [&](int s) -> float {
-    if (S <= 64) return wgt_s[s];
-    const float m = p.part_ml[(((int64_t)bt * S + s) * H + h) * 2];
+    const float a = __shfl_sync(0xffffffffu, w0, s & 31);
+    const float b = __shfl_sync(0xffffffffu, w1, s & 31);
+    if (s < 64) return s < 32 ? a : b;
+    if (s >= S) return 0.f;
+    const float m = ml[(int64_t)s * H].x;
     return m == -INFINITY ? 0.f : exp2f(m - M);
   };
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = grp;; s0 += kR * kCombGroups) {
+  for (int s0 = 0;; s0 += 4 * kR) {
 #pragma unroll
     for (int k = 0; k < kR; ++k) {
-      const int s = s0 + k * kCombGroups;
-      const float w = s < S ? weight(s) : 0.f;
-      acc.x += w * __uint_as_float(v[k].x); acc.y += w * __uint_as_float(v[k].y);
-      acc.z += w * __uint_as_float(v[k].z); acc.w += w * __uint_as_float(v[k].w);
+      const int s = s0 + g + 4 * k;
+      const float w = weight(s);
+      if (s < S) {
+        acc.x += w * __uint_as_float(v[k].x); acc.y += w * __uint_as_float(v[k].y);
+        acc.z += w * __uint_as_float(v[k].z); acc.w += w * __uint_as_float(v[k].w);
+      }
     }
-    if (s0 + kR * kCombGroups >= S) break;
+    if (s0 + 4 * kR >= S) break;
 #pragma unroll
     for (int k = 0; k < kR; ++k) {
-      const int s = s0 + (kR + k) * kCombGroups;
+      const int s = s0 + 4 * kR + g + 4 * k;
       v[k] = s < S ? ld_nc_v4(po + s * sstride) : make_uint4(0, 0, 0, 0);
     }
   }
-  if (grp > 0) part[grp - 1][t] = acc;
-  __syncthreads();
-  if (grp == 0) {
 #pragma unroll
-    for (int g = 0; g < kCombGroups - 1; ++g) {
-      const float4 o = part[g][t];
-      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
-    }
-    const float inv = inv_s;
+  for (int o = 8; o < 32; o <<= 1) {
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o); acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o); acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  if (t == 0 && blockIdx.z == 0 && p.lse) p.lse[(int64_t)bt * H + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+  if (g == 0) {
     const float* cs = p.rope_cs ? p.rope_cs + (int64_t)bt * 64 : nullptr;
     store_out4(p.out, p.out_bf16, ((int64_t)bt * H + h) * kD + d,
                rope_out4(make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv), cs, d));
@@ -535,7 +518,7 @@ static cudaError_t launch_attn_h(AttnParams& p, cudaStream_t stream) {
   note_launches(1);
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    launch_k(attn_combine_kernel, dim3(dim3(p.B * p.n_q, H)), dim3(kCombThreads), 0, stream, p);
+    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, H, kCombChunks), dim3(kCombThreads), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();
@@ -571,7 +554,7 @@ static cudaError_t launch_attn_tc_any(AttnParams& p, const void* q2, cudaStream_
   if (e != cudaSuccess) return e;
   if (p.n_splits > 1) {
     ProfScope ps(stream, "attn_combine");
-    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, p.H), dim3(kCombThreads), 0, stream, p);
+    launch_k(attn_combine_kernel, dim3(p.B * p.n_q, p.H, kCombChunks), dim3(kCombThreads), 0, stream, p);
     note_launches(1);
   }
   return cudaGetLastError();
