@@ -711,6 +711,7 @@ def run_secondary(args, dev, peaks):
                 rec["scorer"] = {"kernel": "index_score_mx", "launch_ms": round(tot / nl, 4), "bytes": kb,
                                  "gbs": round(kb / (tot / nl * 1e-3) / 1e9, 1),
                                  "hbm_frac": round(kb / (tot / nl * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                                 "traffic": _traffic_record("index_score_mx"),
                                  "note": "68 B per key (64 code + 4 exponent bytes); one eager launch with events"}
         out[name] = rec
         del dc, descs, ws
