@@ -89,6 +89,31 @@ def test_index_rejects_bad_args_on_host(csa):
     assert csa._index(ok, None, 0, None) == csa.CSA_ERR_WORKSPACE
 
 
+def test_mx_index_rejects_bad_args_on_host(csa):
+    """MXFP4 keys: 32 heads x 128, the exponent plane 4-byte aligned, and the
+    code plane 32-byte aligned with 32-byte multiple strides (the packed 4-bit
+    copy into the tensor cores' operand layout needs both)."""
+    a = csa.IndexArgs()
+    a.B, a.n_q, a.T, a.H_I, a.d_I, a.K = 2, 1, 1000, 32, 128, 64
+    a.keys = a.q = a.w = a.idx = 4096
+    a.key_row_stride, a.key_batch_stride = 64, 64000
+    a.key_format = csa.CSA_KEY_MXFP4
+    a.key_scales, a.key_scale_row_stride, a.key_scale_batch_stride = 8192, 4, 4000
+    ok = ctypes.byref(a)
+    assert csa._index_ws(ok) > 0
+    assert csa._index(ok, None, 0, None) == csa.CSA_ERR_WORKSPACE      # valid up to the workspace
+    for field, val, want in [("keys", 4096 + 16, csa.CSA_ERR_ALIGNMENT),
+                             ("key_row_stride", 80, csa.CSA_ERR_ALIGNMENT),
+                             ("key_batch_stride", 64016, csa.CSA_ERR_ALIGNMENT),
+                             ("key_scale_row_stride", 6, csa.CSA_ERR_ALIGNMENT),
+                             ("key_scales", None, csa.CSA_ERR_INVALID_ARG),
+                             ("H_I", 8, csa.CSA_ERR_SHAPE), ("d_I", 64, csa.CSA_ERR_SHAPE),
+                             ("n_q", 2, csa.CSA_ERR_UNSUPPORTED)]:
+        b = csa.IndexArgs.from_buffer_copy(a)
+        setattr(b, field, val)
+        assert csa._index(ctypes.byref(b), None, 0, None) == want, field
+
+
 def test_attn_rejects_bad_args_on_host(csa):
     a = csa.AttnArgs()
     a.B, a.n_q, a.H, a.D, a.K, a.n_win = 1, 1, 64, 512, 16, 8
