@@ -118,12 +118,15 @@ index_score_mx_kernel(const __grid_constant__ CUtensorMap tmap, MxScoreParams p)
 
   if (warp == 0) {
     if (lane == 0) {
+      int issued = 0;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % kMxStages;
         if (!mbar_wait(empty + s, ((uint32_t)(i / kMxStages) & 1u) ^ 1u, &g_mx_error, kErrWaitSmemEmpty)) break;
         mbar_arrive_expect_tx(full + s, kMxStageTx);
         tma_load_3d(stage + (size_t)s * kMxStageBytes, &tmap, full + s, 0, (int)((tile0 + i) * kMxRows), b);
+        issued = i + 1;
       }
+      drain_copies(full, kMxStages, issued, &g_mx_error, kErrWaitTmaFull);
     }
   } else if (warp == 1) {
     if (lane == 0) {

@@ -159,6 +159,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
 
   // running tile counter across items keeps the barrier phases consistent
   int64_t run = 0;
+  int64_t issued = 0;                  // key-tile copies issued (producer lane)
   bool failed = false;                 // this thread saw a wait time out
   __shared__ int any_failed;           // block-uniform copy, read after barriers
   __shared__ uint32_t s_cnt[kPfQPerBlock];
@@ -194,6 +195,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
           mbar_arrive_expect_tx(&S.full[s], kPfStageBytes);
           tma_load_3d(S.stage + (size_t)s * kPfStageBytes, &tmap, &S.full[s], 0,
                       (int)(pf_tile(p, x, i) * kPfRows), x.b);
+          issued = g + 1;
         }
       }
     } else if (warp == 1) {
@@ -306,6 +308,7 @@ prefill_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, PfParams p) {
     }
     if (any_failed) break;
   }
+  if (warp == 0 && lane == 0) drain_copies(S.full, kPfStages, issued, &g_pf_error, kErrWaitTmaFull);
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

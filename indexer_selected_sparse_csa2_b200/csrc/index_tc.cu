@@ -122,6 +122,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
   if (warp == 0) {
     if (lane == 0) {
       bool waited = !pre;
+      int issued = 0;
       for (int i = 0; i < n_my; ++i) {
         const int s = i % kTcStages;
         const uint32_t ph = (uint32_t)(i / kTcStages) & 1u;
@@ -132,7 +133,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tmap, TcScoreParams p)
         if (!mbar_wait(&S.empty[s], ph ^ 1u, &g_tc_error, kErrWaitSmemEmpty)) break;
         mbar_arrive_expect_tx(&S.full[s], kTcStageBytes);
         tma_load_3d(S.stage + (size_t)s * kTcStageBytes, &tmap, &S.full[s], 0, (int)((tile0 + i) * kTcRows), b);
+        issued = i + 1;
       }
+      drain_copies(S.full, kTcStages, issued, &g_tc_error, kErrWaitTmaFull);
     }
   } else if (warp == 1) {
     if (lane == 0) {

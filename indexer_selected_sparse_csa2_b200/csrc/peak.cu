@@ -103,6 +103,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ 
           tma_load_2d(sb + (size_t)s * kGmBBytes, &tb, full + s, kb * kGmKB, tn * kGmN);
         }
       }
+      drain_copies(full, kGmStages, it, &g_pk_error, kErrWaitTmaFull);
     }
   } else if (warp == 1) {
     if (lane == 0) {

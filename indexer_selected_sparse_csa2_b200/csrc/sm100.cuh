@@ -68,6 +68,17 @@ CSA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* flag, int code) {
   }
 }
 
+// Bounded wait, by the thread that issued them, for its last copies into a
+// ring of `stages` full-barriers (copy k of [0, issued) went to stage
+// k % stages in phase k / stages).  After a wait that gave up elsewhere the
+// consumer may never have waited for them, and a CTA must not leave while a
+// copy into its shared memory is in flight; phases the consumer already saw
+// complete at once.
+CSA_DEV void drain_copies(uint64_t* full, int stages, int64_t issued, int* flag, int code) {
+  for (int64_t k = issued > stages ? issued - stages : 0; k < issued; ++k)
+    mbar_wait(full + (k % stages), (uint32_t)(k / stages) & 1u, flag, code);
+}
+
 // --------------------------------------------------------------------- TMA --
 CSA_DEV void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(
