@@ -1,11 +1,11 @@
 // sm_100a building blocks: mbarriers with bounded waits, TMA tensor loads,
 // tcgen05 MMA / TMEM, shared-memory and instruction descriptors.
 //
-// Written against the PTX ISA for sm_100a.  No TMA load here uses cluster
-// multicast.  Every wait is bounded in wall-clock time: after kWaitNs
-// nanoseconds (%globaltimer) it records an error code in a device flag (read
-// by csa_device_status()) and returns false, so a kernel can never spin
-// forever.
+// Written against the PTX ISA for sm_100a.  Every TMA load here fills the
+// issuing CTA's own shared memory only.  Every wait is bounded in wall-clock
+// time: after kWaitNs nanoseconds (%globaltimer) it records an error code in
+// a device flag (read by csa_device_status()) and returns false, so a kernel
+// can never spin forever.
 #pragma once
 
 #include <cuda.h>
@@ -100,7 +100,7 @@ CSA_DEV void cp_async16(uint32_t dst_smem, const void* src) {
 }
 CSA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 CSA_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-// Untiled bulk copy global -> this CTA's shared memory (no multicast):
+// Untiled bulk copy global -> this CTA's own shared memory:
 // addresses 16-byte aligned, bytes a multiple of 16; completes on `bar`.
 CSA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
